@@ -1,0 +1,35 @@
+"""Planted mistakes in the oracle must be caught by its pins.
+
+Each variant is the oracle source compiled with one ``-DORACLE_MUTANT_*``
+macro (a swapped nibble order, a dropped min term, ties rounded away from
+zero, an off-by-one block sum, a shifted group index, a dropped block-sum
+term in the W4A8 product).  The mistake lives in the oracle on the CPU; no GPU
+code is involved.  Every variant must fail at least one pin.
+"""
+import pytest
+
+import oracle
+import oracle_pins
+
+MUTANTS = [
+    "SWAP_NIBBLES",
+    "DROP_MIN",
+    "ROUND_AWAY",
+    "BLOCKSUM_OFF_BY_ONE",
+    "GROUP_INDEX",
+    "MMQ_DROP_BLOCKSUM",
+]
+
+
+@pytest.mark.parametrize("mutant", MUTANTS)
+def test_mutant_is_caught(tmp_path, mutant):
+    path = oracle.compile_oracle(str(tmp_path / f"liboracle_{mutant}.so"),
+                                 defines=(f"ORACLE_MUTANT_{mutant}",), openmp=False)
+    o = oracle.Oracle(oracle.load(path))
+    failed = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(o)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught the planted mistake {mutant}"
