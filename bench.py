@@ -1,0 +1,600 @@
+#!/usr/bin/env python3
+"""Benchmark of the W4-G256 quantized-matmul hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Timed step (the workload the headline metric is quoted on): the batch-1
+decode GEMV sweep over the five 4B-class shapes
+    (N,K) = (6144,2560) (2560,4096) (19456,2560) (2560,9728) (151936,2560),
+W4-G256 weights quantised on the device from fp32 N(0, 0.02), x ~ N(0,1) bf16,
+bf16 output.  Two weight copies alternate between steps (505 MB, four times
+the 126 MB L2), so every step streams its weights from HBM.
+
+value = algorithmic bytes of all five GEMVs (codes + scales + x + y) per step
+x steps / device time, in GB/s, summed over ranks (replicas; weak scaling).
+Also measured in the same run (reported under their own keys): the small-batch
+sweep (M = 2, 4, 8), the W4A8 prefill product (M = 256..2048 on both prefill
+shapes, TOPS), the activation quantiser (GB/s) and the graph-captured
+per-token chain (36 layers x 4 shapes + lm_head, tok/s-equivalent).
+
+One JSON line is printed by rank 0.  `--impl reference` times the CPU oracle
+on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W4 GEMV HBM GB/s at batch 1; W4A8 MMQ prefill TOPS; % of roofline"
+SHAPES = synth.GEMV_SHAPES
+GROUP = 256
+# Nominal dense int8 / bf16 tensor ratio (4.5 / 2.25 PFLOP/s): the int8 peak
+# used for the prefill product is the measured bf16 peak times this ratio.
+INT8_OVER_BF16 = 2.0
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+# ---------------------------------------------------------------------------
+
+def gemv_bytes(N: int, K: int, M: int, out_bytes: int = 2) -> int:
+    """Bytes a GEMV must move at least once: codes, d, m, x and y."""
+    return N * K // 2 + N * (K // GROUP) * 4 + M * K * 2 + M * N * out_bytes
+
+
+def mmq_ops(M: int, N: int, K: int) -> int:
+    return 2 * M * N * K
+
+
+def mmq_bytes(M: int, N: int, K: int) -> int:
+    return N * K // 2 + N * (K // GROUP) * 4 + M * K + M * (K // 32) * 8 + M * N * 2
+
+
+def quant_bytes(M: int, K: int) -> int:
+    return M * K * 2 + M * K + M * (K // 32) * 8
+
+
+# ---------------------------------------------------------------------------
+# environment helpers
+# ---------------------------------------------------------------------------
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def source_hash(*files: str) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(key)
+    if not e or e.get("source_hash") != source_hash(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread:
+                self.thread.join(timeout=2)
+
+    def summary(self) -> dict:
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_timing(elapsed_s: float, units: float, device=None):
+    """Max of elapsed time and sum of work units over ranks (identity on one
+    process).  Every rank must call it the same number of times."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return elapsed_s, units
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+class Workload:
+    """Device-resident weights (two copies per shape) and activations."""
+
+    def __init__(self, torch, w4, dev, copies=2, seed=7):
+        self.torch, self.w4, self.dev = torch, w4, dev
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        self.weights = []  # [copy][shape] -> (codes, d, m)
+        for c in range(copies):
+            per = []
+            for (N, K) in SHAPES:
+                w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32)
+                w.mul_(0.02)
+                per.append(w4.w4_pack(w))
+                del w
+            self.weights.append(per)
+        torch.cuda.synchronize()
+        self.x = {}
+        self.y = {}
+
+    def xs(self, M):
+        if M not in self.x:
+            torch = self.torch
+            self.x[M] = [torch.from_numpy(synth.activations(M, K, synth.act_seed(
+                synth.CONFIG_BATCH1 if M == 1 else synth.CONFIG_SMALL_BATCH, i)).view(np.int16))
+                .to(self.dev).view(torch.bfloat16) for i, (N, K) in enumerate(SHAPES)]
+            self.y[M] = [torch.empty((M, N), dtype=torch.bfloat16, device=self.dev)
+                         for (N, K) in SHAPES]
+        return self.x[M], self.y[M]
+
+
+def time_gemv_sweep(torch, w4, wl, M, steps, warmup, stream, dom_index=4):
+    """Times `steps` sweeps; returns (elapsed_s, per-shape mean ms, launches)."""
+    xs, ys = wl.xs(M)
+    ncopy = len(wl.weights)
+
+    def step(i, ev=None):
+        wset = wl.weights[i % ncopy]
+        for s in range(len(SHAPES)):
+            codes, d, m = wset[s]
+            if ev is not None:
+                ev[s][0].record(stream)
+            w4.w4_gemv(codes, d, m, xs[s], out_dtype=torch.bfloat16, y=ys[s], stream=stream)
+            if ev is not None:
+                ev[s][1].record(stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    # pass 1: the whole timed region, bracketed by events only
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        step(i)
+    end.record(stream)
+    torch.cuda.synchronize()
+    elapsed = start.elapsed_time(end) / 1e3
+    # pass 2: per-launch events on the launching stream (per-kernel times)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in SHAPES]
+           for _ in range(steps)]
+    for i in range(steps):
+        step(i, evs[i])
+    torch.cuda.synchronize()
+    per = [statistics.mean(evs[i][s][0].elapsed_time(evs[i][s][1]) for i in range(steps))
+           for s in range(len(SHAPES))]
+    return elapsed, per, steps * len(SHAPES)
+
+
+def time_e2e(torch, w4, wl, steps, warmup, stream):
+    """Same sweep through host buffers: pinned x -> device, GEMVs, y -> host."""
+    M = 1
+    xs_h = [torch.from_numpy(synth.activations(M, K, synth.act_seed(synth.CONFIG_BATCH1, i))
+                             .view(np.int16)).view(torch.bfloat16).pin_memory()
+            for i, (N, K) in enumerate(SHAPES)]
+    ys_h = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for (N, K) in SHAPES]
+    xs_d = [x.to(wl.dev) for x in xs_h]
+    ys_d = [torch.empty((M, N), dtype=torch.bfloat16, device=wl.dev) for (N, K) in SHAPES]
+    ncopy = len(wl.weights)
+
+    def step(i):
+        for s in range(len(SHAPES)):
+            codes, d, m = wl.weights[i % ncopy][s]
+            xs_d[s].copy_(xs_h[s], non_blocking=True)
+            w4.w4_gemv(codes, d, m, xs_d[s], out_dtype=torch.bfloat16, y=ys_d[s], stream=stream)
+            ys_h[s].copy_(ys_d[s], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            step(i)
+        torch.cuda.synchronize()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(steps):
+            step(i)
+        end.record(stream)
+        torch.cuda.synchronize()
+    h2d = sum(x.numel() * 2 for x in xs_h)
+    d2h = sum(y.numel() * 2 for y in ys_h)
+    return start.elapsed_time(end) / 1e3, h2d, d2h
+
+
+def time_mmq(torch, w4, dev, stream, reps=5):
+    """W4A8 prefill product at M = 256..2048 on both prefill shapes, plus the
+    activation quantiser.  Returns a list of result dicts."""
+    out = []
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for si, (N, K) in enumerate(synth.MMQ_SHAPES):
+        w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
+        codes, d, m = w4.w4_pack(w)
+        del w
+        for M in synth.MMQ_M:
+            x = torch.from_numpy(synth.outlier_activations(M, K, synth.act_seed(
+                synth.CONFIG_MMQ, si)).view(np.int16)).to(dev).view(torch.bfloat16)
+            qa, dx, S = w4.q8_quantize_act(x, stream=stream)
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            for _ in range(3):
+                w4.w4a8_mmq(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y, stream=stream)
+            tq, tm = [], []
+            for _ in range(reps):
+                flush.zero_()
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+                w4.q8_quantize_act(x, qa, dx, S, stream=stream)
+                e1.record(stream)
+                w4.w4a8_mmq(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y, stream=stream)
+                e2.record(stream)
+                torch.cuda.synchronize()
+                tq.append(e0.elapsed_time(e1) / 1e3)
+                tm.append(e1.elapsed_time(e2) / 1e3)
+            t_mmq = statistics.median(tm)
+            t_q = statistics.median(tq)
+            out.append({"M": M, "N": N, "K": K, "mmq_us": t_mmq * 1e6,
+                        "tops": mmq_ops(M, N, K) / t_mmq / 1e12,
+                        "quant_us": t_q * 1e6, "quant_gbs": quant_bytes(M, K) / t_q / 1e9,
+                        "mmq_min_us": min(tm) * 1e6, "mmq_max_us": max(tm) * 1e6})
+            del x, qa, dx, S, y
+    del flush
+    return out
+
+
+def time_chain(torch, w4, dev, stream, reps=5):
+    """36 layers x 4 layer shapes + lm_head, M = 1, distinct weights per layer,
+    captured once in a CUDA graph and replayed."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(13)
+    layers = []
+    for _ in range(synth.CHAIN_LAYERS):
+        per = []
+        for (N, K) in synth.LAYER_SHAPES:
+            w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
+            per.append(w4.w4_pack(w))
+            del w
+        layers.append(per)
+    N, K = synth.LM_HEAD
+    w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
+    head = w4.w4_pack(w)
+    del w
+    xs = [torch.randn((1, K), generator=g, device=dev).to(torch.bfloat16)
+          for (N, K) in synth.LAYER_SHAPES + [synth.LM_HEAD]]
+    ys = [torch.empty((1, N), dtype=torch.bfloat16, device=dev)
+          for (N, K) in synth.LAYER_SHAPES + [synth.LM_HEAD]]
+    total = (synth.CHAIN_LAYERS * sum(gemv_bytes(N, K, 1) for N, K in synth.LAYER_SHAPES)
+             + gemv_bytes(*synth.LM_HEAD, 1))
+
+    def chain():
+        for L in layers:
+            for s, (codes, d, m) in enumerate(L):
+                w4.w4_gemv(codes, d, m, xs[s], out_dtype=torch.bfloat16, y=ys[s],
+                           stream=torch.cuda.current_stream())
+        w4.w4_gemv(*head, xs[4], out_dtype=torch.bfloat16, y=ys[4],
+                   stream=torch.cuda.current_stream())
+
+    with torch.cuda.stream(stream):
+        chain()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            chain()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(ts)
+    del graph
+    return {"tok_per_s": 1.0 / t, "ms_per_token": t * 1e3, "gbs": total / t / 1e9,
+            "bytes_per_token": total, "launches": synth.CHAIN_LAYERS * 4 + 1}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=datetime.timedelta(seconds=120))
+    import w4_quant_matmul_b200 as w4
+    peaks = load_peaks()
+    stream = torch.cuda.Stream(device=dev)
+    wl = Workload(torch, w4, dev)
+    step_bytes = sum(gemv_bytes(N, K, 1) for N, K in SHAPES)
+
+    # --- timed region: K steps of the batch-1 sweep ---
+    barrier(dev)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        elapsed, per_shape_ms, launches = time_gemv_sweep(torch, w4, wl, 1, args.steps,
+                                                          args.warmup, stream)
+    barrier(dev)
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    elapsed_max, bytes_all = reduce_timing(elapsed, step_bytes * args.steps, dev)
+    value = bytes_all / elapsed_max / 1e9
+
+    # dominant kernel: the lm_head GEMV (largest stream, ~80% of the step)
+    N, K = SHAPES[4]
+    dom_bytes = gemv_bytes(N, K, 1)
+    dom_s = per_shape_ms[4] / 1e3
+    achieved = dom_bytes / dom_s / 1e9
+    traffic = load_traffic("w4_quant_matmul_b200/csrc/gemv.cu", "w4_gemv_lm_head_m1")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "kernel": "w4_gemv_kernel (151936x2560, M=1)",
+                "algorithmic_bytes": dom_bytes,
+                "peak_source": f"{peaks['source']} hbm_gbs"}
+
+    # --- e2e through host buffers ---
+    t_e2e, h2d, d2h = time_e2e(torch, w4, wl, args.steps, args.warmup, stream)
+    t_e2e_max, bytes_e2e = reduce_timing(t_e2e, step_bytes * args.steps, dev)
+    e2e = {"value": round(bytes_e2e / t_e2e_max / 1e9, 1), "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    extras = {}
+    per_shape = [{"N": n, "K": k, "us": ms * 1e3,
+                  "gbs": round(gemv_bytes(n, k, 1) / (ms / 1e3) / 1e9, 1)}
+                 for (n, k), ms in zip(SHAPES, per_shape_ms)]
+    extras["gemv_m1"] = per_shape
+    if not args.quick:
+        for M in synth.SMALL_BATCH:
+            e, per, _ = time_gemv_sweep(torch, w4, wl, M, max(3, args.steps // 2), 2, stream)
+            extras[f"gemv_m{M}"] = [{"N": n, "K": k, "us": round(ms * 1e3, 2),
+                                     "gbs": round(gemv_bytes(n, k, M) / (ms / 1e3) / 1e9, 1),
+                                     "tok_per_s": round(M / (ms / 1e3), 1)}
+                                    for (n, k), ms in zip(SHAPES, per)]
+        del wl
+        torch.cuda.empty_cache()
+        mmq = time_mmq(torch, w4, dev, stream)
+        int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+        for r in mmq:
+            r["frac_int8_peak"] = round(r["tops"] / int8_peak, 4)
+            r["frac_datasheet_4500"] = round(r["tops"] / 4500.0, 4)
+        extras["mmq"] = mmq
+        extras["int8_peak_tops"] = {"value": int8_peak,
+                                    "how": f"{peaks['source']} bf16 burst x {INT8_OVER_BF16}"}
+        torch.cuda.empty_cache()
+        extras["chain"] = time_chain(torch, w4, dev, stream)
+        extras["chain"]["frac_hbm"] = round(extras["chain"]["gbs"] / peaks["hbm_gbs"], 4)
+    w4.w4_check_device_error()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(seconds=args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(elapsed_max / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u4 codes x bf16 (fp32 accumulate)", "data": "synthetic",
+            "config": {"workload": "batch-1 decode GEMV sweep, W4-G256, (N,K) = "
+                                   "(6144,2560) (2560,4096) (19456,2560) (2560,9728) "
+                                   "(151936,2560), M=1, bf16 out",
+                       "global_batch": world, "seq_len": 1,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2: two 253 MB weight sets alternate"},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk.summary(), "cpu_baseline": cpu,
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier(dev)
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle arm
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(rows_per_shape: int):
+    """Oracle-packed weights for the first `rows_per_shape` rows of each shape
+    (fp32 N(0, 0.02) from the same generator family) and the M = 1 x."""
+    import oracle
+    o = oracle.get()
+    sample = []
+    for i, (N, K) in enumerate(SHAPES):
+        n = min(N, rows_per_shape)
+        w = synth.dense_weights(n, K, synth.weight_seed(synth.CONFIG_BATCH1, i))
+        codes, d, m = o.w4_pack(w)
+        x = synth.activations(1, K, synth.act_seed(synth.CONFIG_BATCH1, i))
+        sample.append((codes, d, m, x, n, K))
+    return o, sample
+
+
+def cpu_baseline(seconds: float = 15.0, rows_per_shape: int = 2048) -> dict:
+    """The oracle GEMV (fp64, OpenMP over rows) on a bounded sample of the
+    batch-1 sweep, timed on this host's cores."""
+    o, sample = _oracle_sample(rows_per_shape)
+    nbytes = sum(gemv_bytes(n, K, 1) for (_, _, _, _, n, K) in sample)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for codes, d, m, x, n, K in sample:
+            o.gemv(codes, d, m, x)
+        reps += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(nbytes * reps / dt / 1e9, 3), "unit": "GB/s",
+            "cores": o.num_threads(), "kind": "oracle",
+            "sample": f"{rows_per_shape} rows of each of the 5 batch-1 shapes (M=1), "
+                      f"{reps} passes, {dt:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    o, sample = _oracle_sample(2048)
+    nbytes = sum(gemv_bytes(n, K, 1) for (_, _, _, _, n, K) in sample)
+
+    def step():
+        for codes, d, m, x, n, K in sample:
+            o.gemv(codes, d, m, x)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = nbytes * args.steps / dt / 1e9
+    sample_desc = "2048 rows of each of the 5 batch-1 shapes (M=1) per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "batch-1 decode GEMV sweep, W4-G256 (CPU oracle sample)",
+                   "global_batch": 1, "seq_len": 1, "parallelism": "cpu"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": o.num_threads(),
+                         "kind": "oracle", "sample": sample_desc},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--quick", action="store_true", help="only the timed batch-1 sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

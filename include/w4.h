@@ -1,0 +1,152 @@
+/*
+ * w4.h -- C ABI of libw4, the B200 (sm_100a) W4-G256 quantized-matmul library.
+ *
+ * Format (W4-G256; "HFQ4-G256" in the hipfire MMQ prefill article):
+ *   W[N,K], K a multiple of 256, split into groups of 256 consecutive k per
+ *   row.  Each group stores 128 bytes of 4-bit codes q in [0,15] plus an fp16
+ *   scale d and an fp16 min m; a weight dequantises to w = d*q + m.
+ *   Storage is three dense row-major planes:
+ *     codes  uint8 [N][K/2]  byte j of a row holds k = 2j in bits 0-3 and
+ *                            k = 2j+1 in bits 4-7
+ *     d      fp16  [N][K/256] (raw IEEE binary16 bits)
+ *     m      fp16  [N][K/256]
+ *   Activations are bf16 [M][K] row-major (raw bits).  For the W4A8 product
+ *   they are first quantised per 32-element block (the Q8_1-style MMQ layout
+ *   the article pre-quantises prefill activations to):
+ *     qa  int8  [M][K]      codes in [-127,127]
+ *     dx  fp32  [M][K/32]   block scale amax/127 (0 for an all-zero block)
+ *     S   int32 [M][K/32]   sum of the block's qa
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers to caller-owned memory.  The
+ *     library never allocates, frees or synchronises; it only enqueues work on
+ *     `stream` (a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream) and returns.
+ *   - Base pointers must be 16-byte aligned; row strides are the dense ones
+ *     implied by the shapes above.
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     violation returns its status and enqueues nothing.
+ *   - The device must be a compute-capability 10.0 GPU (B200 class); any other
+ *     device gives W4_ERR_UNSUPPORTED_DEVICE.  There is no fallback path.
+ *   - W4_ERR_CUDA reports a launch error; w4_last_cuda_error() gives the CUDA
+ *     error code.  Inputs are assumed finite (not checked).
+ *   - Every kernel waits for its own pipeline with bounded spins; a wait that
+ *     runs out sets a device-side error word and the kernel returns early.
+ *     w4_check_device_error() reads (and clears) that word.
+ *   - Results are bitwise deterministic run to run (fixed reduction orders, no
+ *     floating-point atomics).
+ */
+#ifndef W4_H
+#define W4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W4_ABI_VERSION 1
+
+typedef enum {
+    W4_OK = 0,
+    W4_ERR_NULL = 1,               /* a required pointer is NULL            */
+    W4_ERR_SHAPE = 2,              /* a size violates the format or range   */
+    W4_ERR_ALIGN = 3,              /* a base pointer is not 16-byte aligned */
+    W4_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100          */
+    W4_ERR_WORKSPACE = 5,          /* workspace missing or too small        */
+    W4_ERR_CUDA = 6,               /* a CUDA call or launch failed          */
+    W4_ERR_TIMEOUT = 7             /* a kernel's bounded wait ran out       */
+} w4_status;
+
+typedef enum {
+    W4_OUT_BF16 = 0, /* y stored as bf16, round to nearest even of the fp32 sum */
+    W4_OUT_F32 = 1   /* y stored as fp32                                        */
+} w4_out_dtype;
+
+/* ABI version of the loaded library (W4_ABI_VERSION at build time). */
+int w4_abi_version(void);
+
+/* Static, human-readable name of a status code. */
+const char *w4_status_string(int status);
+
+/* CUDA error code (cudaError_t as int) behind the last W4_ERR_CUDA on this
+ * host thread, or 0. */
+int w4_last_cuda_error(void);
+
+/* Synchronises the current device, then returns W4_ERR_TIMEOUT if any kernel
+ * of this library gave up a bounded wait since the last call (and clears the
+ * flag), W4_ERR_CUDA if the synchronisation failed, else W4_OK. */
+int w4_check_device_error(void);
+
+/* Quantise and pack fp32 weights, min/max per group of 256.
+ * Defined by: the format definition above ("groups of 256 ... 4-bit codes
+ * plus fp16 d and fp16 m, w = d*q + m"); the rounding rule is the reading
+ * adopted where the pages are silent:
+ *   per (row, group): mn, mx = min, max (fp32);
+ *   d16 = fp16_rn((mx - mn) / 15); m16 = fp16_rn(mn);
+ *   q = 0 if d16 == 0 else clamp(rint((w - m16) / d16), 0, 15), ties to even,
+ *   all arithmetic IEEE fp32 round-to-nearest.
+ * w: fp32 [N][K]; outputs codes [N][K/2], d [N][K/256], m [N][K/256].
+ * N >= 0, K >= 0, K % 256 == 0.  N == 0 or K == 0 enqueues nothing. */
+int w4_pack(const float *w, int64_t N, int64_t K, uint8_t *codes,
+            uint16_t *d_f16, uint16_t *m_f16, void *stream);
+
+/* Pack one-code-per-byte q [N][K] (values 0..15; higher bits are ignored)
+ * into codes [N][K/2] with the nibble order above.  K % 2 == 0 and
+ * (N*K) % 32 == 0. */
+int w4_pack_codes(const uint8_t *q, int64_t N, int64_t K, uint8_t *codes,
+                  void *stream);
+
+/* Inverse of w4_pack_codes: codes [N][K/2] -> q [N][K], one code per byte.
+ * K % 2 == 0 and (N*K) % 32 == 0. */
+int w4_unpack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *q,
+              void *stream);
+
+/* Decode GEMV, dequantisation fused into the weight stream (the batch-1
+ * decode "quant-GEMM bandwidth ladder" of the GFX1100-TG150/TG200 pages):
+ *   y[t][n] = sum_g ( d[n][g] * sum_{k in g} q[n][k] * x[t][k]
+ *                     + m[n][g] * sum_{k in g} x[t][k] )
+ * for t < M, n < N, accumulated in fp32.
+ * codes/d/m: the format planes of W[N][K]; x: bf16 [M][K]; y: [M][N] of
+ * out_dtype.  1 <= M <= 8, N >= 1, K >= 256, K % 256 == 0. */
+int w4_gemv(const uint8_t *codes, const uint16_t *d_f16,
+            const uint16_t *m_f16, int64_t N, int64_t K,
+            const uint16_t *x_bf16, int M, void *y, int out_dtype,
+            void *stream);
+
+/* Quantise bf16 activations to int8 per block of 32 (the article's
+ * "pre-quantise prefill activations to the Q8_1 MMQ layout"), with the
+ * reading adopted for the unprinted rule:
+ *   amax = max |x|;  dx = amax / 127 (IEEE fp32 division);
+ *   amax == 0 -> dx = 0, qa = 0, S = 0;
+ *   else qa = clamp(rint(x / dx), -127, 127), ties to even;  S = sum(qa).
+ * x: bf16 [M][K] -> qa int8 [M][K], dx fp32 [M][K/32], S int32 [M][K/32].
+ * M >= 0, K % 32 == 0. */
+int q8_quantize_act(const uint16_t *x_bf16, int64_t M, int64_t K, int8_t *qa,
+                    float *dx, int32_t *bsum, void *stream);
+
+/* Bytes of device workspace w4a8_mmq needs for this shape (0 means none; the
+ * workspace pointer may then be NULL). */
+size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* W4A8 prefill product on int8 tensor cores (the article's MMQ path: int8
+ * activations, tiled int8 matrix-matrix over the 4-bit weights, scales
+ * applied after the integer products):
+ *   P[t][n][b] = sum_{k in block b} q[n][k] * qa[t][k]      (exact int32)
+ *   y[t][n]    = sum_g ( d[n][g] * sum_{b in g} dx[t][b] * P[t][n][b]
+ *                        + m[n][g] * sum_{b in g} dx[t][b] * S[t][b] )
+ * scales applied in fp32.  codes/d/m: W[N][K] planes; qa/dx/bsum: the
+ * output of q8_quantize_act for x [M][K]; y: [M][N] of out_dtype.
+ * M >= 1, N >= 1, K >= 256, K % 256 == 0.  `workspace` must hold
+ * w4a8_mmq_workspace_size(M, N, K) bytes. */
+int w4a8_mmq(const uint8_t *codes, const uint16_t *d_f16,
+             const uint16_t *m_f16, int64_t N, int64_t K, const int8_t *qa,
+             const float *dx, const int32_t *bsum, int64_t M, void *y,
+             int out_dtype, void *workspace, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4_H */

@@ -1,0 +1,124 @@
+"""The C ABI: the built library loads and exports every entry point that
+include/w4.h declares; argument validation answers before anything touches a
+device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4_quant_matmul_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_0-9]+)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for expected in ["w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "q8_quantize_act",
+                     "w4a8_mmq", "w4a8_mmq_workspace_size", "w4_status_string",
+                     "w4_abi_version", "w4_last_cuda_error", "w4_check_device_error"]:
+        assert expected in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_binding_covers_every_declared_symbol():
+    from w4_quant_matmul_b200 import _lib
+    assert set(declared_functions()) == set(_lib.SIGNATURES)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.w4_abi_version() == 1
+    for code in range(8):
+        s = lib.w4_status_string(code).decode()
+        assert s.startswith("W4_")
+    assert "unknown" in lib.w4_status_string(99).decode()
+
+
+FAKE = 0x10000  # never dereferenced: validation fails first
+MIS = 0x10001   # misaligned
+
+
+def test_gemv_validation(lib):
+    from w4_quant_matmul_b200 import _lib as L
+    f = lib.w4_gemv
+    # shapes first
+    assert f(FAKE, FAKE, FAKE, 256, 300, FAKE, 1, FAKE, 0, None) == L.W4_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, 0, FAKE, 0, None) == L.W4_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, 9, FAKE, 0, None) == L.W4_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, 0, 512, FAKE, 1, FAKE, 0, None) == L.W4_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, 1, FAKE, 7, None) == L.W4_ERR_SHAPE
+    # then pointers
+    assert f(None, FAKE, FAKE, 256, 512, FAKE, 1, FAKE, 0, None) == L.W4_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, 256, 512, None, 1, FAKE, 0, None) == L.W4_ERR_NULL
+    assert f(MIS, FAKE, FAKE, 256, 512, FAKE, 1, FAKE, 0, None) == L.W4_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, 1, MIS, 0, None) == L.W4_ERR_ALIGN
+
+
+def test_pack_and_quantizer_validation(lib):
+    from w4_quant_matmul_b200 import _lib as L
+    assert lib.w4_pack(FAKE, 4, 300, FAKE, FAKE, FAKE, None) == L.W4_ERR_SHAPE
+    assert lib.w4_pack(None, 4, 256, FAKE, FAKE, FAKE, None) == L.W4_ERR_NULL
+    assert lib.w4_pack(FAKE, 4, 256, FAKE, MIS, FAKE, None) == L.W4_ERR_ALIGN
+    assert lib.w4_pack(FAKE, 0, 256, FAKE, FAKE, FAKE, None) == L.W4_OK  # nothing to do
+    assert lib.w4_pack_codes(FAKE, 3, 5, FAKE, None) == L.W4_ERR_SHAPE
+    assert lib.w4_unpack(None, 3, 4, FAKE, None) == L.W4_ERR_NULL
+    assert lib.q8_quantize_act(FAKE, 2, 48, FAKE, FAKE, FAKE, None) == L.W4_ERR_SHAPE
+    assert lib.q8_quantize_act(FAKE, 2, 64, FAKE, None, FAKE, None) == L.W4_ERR_NULL
+    assert lib.q8_quantize_act(FAKE, 2, 64, FAKE, FAKE, MIS, None) == L.W4_ERR_ALIGN
+    assert lib.q8_quantize_act(FAKE, 0, 64, FAKE, FAKE, FAKE, None) == L.W4_OK
+
+
+def test_mmq_validation(lib):
+    from w4_quant_matmul_b200 import _lib as L
+    f = lib.w4a8_mmq
+    args = [FAKE, FAKE, FAKE, 256, 512, FAKE, FAKE, FAKE, 128, FAKE, 0, None, 0, None]
+
+    def call(**kw):
+        a = list(args)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return f(*a)
+
+    assert call(a4=384) == L.W4_ERR_SHAPE          # K % 256
+    assert call(a4=256 * 65) == L.W4_ERR_SHAPE     # K above the supported maximum
+    assert call(a8=0) == L.W4_ERR_SHAPE            # M
+    assert call(a10=3) == L.W4_ERR_SHAPE           # out dtype
+    assert call(a5=None) == L.W4_ERR_NULL
+    assert call(a6=MIS) == L.W4_ERR_ALIGN
+    assert lib.w4a8_mmq_workspace_size(2048, 19456, 2560) == 0
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    from w4_quant_matmul_b200 import _lib as L
+    monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(L, "_lib", None)
+    with pytest.raises(L.LibraryMissing):
+        L.load()
+
+
+def test_product_package_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "w4_quant_matmul_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, fn)).read()
+                assert "oracle" not in src.lower(), fn

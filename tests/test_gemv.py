@@ -1,0 +1,122 @@
+"""w4_gemv on the GPU against the fp64 oracle.
+
+Gate (fp32 output): normwise max relative error <= 2e-3 and NMSE <= 1e-6.
+bf16 output: bitwise RN-bf16 of the same kernel's fp32 output.  Small cases
+compare every output; the full-size decode shapes (M = 1, 2, 4, 8) compare a
+seeded sample of rows, in the launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+
+import parity
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    return parity.cuda_or_skip()
+
+
+@pytest.fixture(scope="module")
+def w4(torch):
+    import w4_quant_matmul_b200 as w4
+    return w4
+
+
+def _dev_u16(torch, a, dtype):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(dtype)
+
+
+def _run(torch, w4, codes, d, m, x_bits, out):
+    y = w4.w4_gemv(torch.from_numpy(codes).cuda(), _dev_u16(torch, d, torch.float16),
+                   _dev_u16(torch, m, torch.float16), _dev_u16(torch, x_bits, torch.bfloat16),
+                   out_dtype=out)
+    torch.cuda.synchronize()
+    if out == torch.float32:
+        return y.cpu().numpy()
+    return y.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _both(torch, w4, orc, codes, d, m, x, rows=None, what=""):
+    y32 = _run(torch, w4, codes, d, m, x, torch.float32)
+    y16 = _run(torch, w4, codes, d, m, x, torch.bfloat16)
+    if rows is None:
+        ref = orc.gemv(codes, d, m, x)
+    else:
+        ref = np.concatenate([orc.gemv(codes, d, m, x, rows=(int(r), int(r) + 1)) for r in rows],
+                             axis=1)
+        y32, y16 = y32[:, rows], y16[:, rows]
+    parity.assert_f32_gate(y32, ref, what)
+    parity.assert_bf16_consistent(y16, y32, ref, what)
+    return y32
+
+
+def test_tiny_case(torch, w4, orc):
+    codes, d, m, x = synth.tiny(0)
+    _both(torch, w4, orc, codes, d, m, x, what="tiny")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("N,K", [(1, 256), (17, 768), (200, 512), (300, 2560), (64, 4608)])
+def test_small_shapes_all_outputs(torch, w4, orc, M, N, K):
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=N + K + M)
+    x = synth.activations(M, K, seed=N * K + M)
+    _both(torch, w4, orc, codes, d, m, x, what=f"M{M} N{N} K{K}")
+
+
+def test_degenerate_weights(torch, w4, orc):
+    N, K = 40, 512
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=5)
+    d[:10] = 0          # scale zero: only the min term
+    m[10:20] = 0        # min zero: only the code term
+    codes[20:30] = 0xFF  # all codes 15
+    x = synth.activations(2, K, seed=6)
+    x[1, :256] = 0      # zero activations in one group
+    _both(torch, w4, orc, codes, d, m, x, what="degenerate")
+
+
+@pytest.mark.parametrize("shape_index", range(len(synth.GEMV_SHAPES)))
+def test_full_size_sampled_rows(torch, w4, orc, shape_index):
+    N, K = synth.GEMV_SHAPES[shape_index]
+    _, codes, d, m = parity.packed_dense_weights(N, K, synth.weight_seed(synth.CONFIG_BATCH1,
+                                                                         shape_index))
+    rows = parity.sample_rows(N)
+    for M in (1, 2, 4, 8):
+        cfg = synth.CONFIG_BATCH1 if M == 1 else synth.CONFIG_SMALL_BATCH
+        x = synth.activations(M, K, synth.act_seed(cfg, shape_index))
+        _both(torch, w4, orc, codes, d, m, x, rows=rows, what=f"{N}x{K} M{M}")
+
+
+def test_deterministic_and_guard_bands(torch, w4):
+    N, K, M = 1000, 2560, 4
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=8)
+    x = synth.activations(M, K, seed=9)
+    dc = torch.from_numpy(codes).cuda()
+    dd = _dev_u16(torch, d, torch.float16)
+    dm = _dev_u16(torch, m, torch.float16)
+    dxx = _dev_u16(torch, x, torch.bfloat16)
+    pad = 64
+    buf = torch.full((M * N + 2 * pad,), 12345.0, dtype=torch.float32, device="cuda")
+    y = buf[pad:pad + M * N].view(M, N)
+    w4.w4_gemv(dc, dd, dm, dxx, out_dtype=torch.float32, y=y)
+    first = y.clone()
+    w4.w4_gemv(dc, dd, dm, dxx, out_dtype=torch.float32, y=y)
+    torch.cuda.synchronize()
+    assert torch.equal(first.view(torch.int32), y.view(torch.int32))
+    assert torch.all(buf[:pad] == 12345.0) and torch.all(buf[pad + M * N:] == 12345.0)
+
+
+def test_rejects_bad_arguments(torch, w4):
+    codes = torch.zeros((16, 128), dtype=torch.uint8, device="cuda")
+    d = torch.zeros((16, 1), dtype=torch.float16, device="cuda")
+    x = torch.zeros((9, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(w4.W4Error):
+        w4.w4_gemv(codes, d, d, x)   # M = 9
+    x = torch.zeros((1, 256), dtype=torch.bfloat16, device="cuda")
+    buf = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    y_mis = buf[1:17][None, :]   # 2-byte offset: not 16-byte aligned
+    with pytest.raises(w4.W4Error):
+        w4.w4_gemv(codes, d, d, x, y=y_mis)
+    w4.w4_check_device_error()

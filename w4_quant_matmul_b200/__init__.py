@@ -1,0 +1,210 @@
+"""W4-G256 quantized matmul for B200 (sm_100a): Python binding.
+
+Every function here marshals torch CUDA tensors into the C ABI of libw4.so
+(``include/w4.h``) and raises ``W4Error`` on a non-OK status.  All arithmetic
+runs in the library's CUDA kernels; torch only provides device memory and the
+current stream.  There is no CPU path: without the built library, calls raise
+``LibraryMissing``.
+
+Entry points (same names as the C ABI):
+    w4_pack(w)                              -> codes, d, m
+    w4_pack_codes(q)                        -> codes
+    w4_unpack(codes, K)                     -> q
+    w4_gemv(codes, d, m, x, out_dtype)      -> y
+    q8_quantize_act(x)                      -> qa, dx, bsum
+    w4a8_mmq(codes, d, m, qa, dx, bsum, out_dtype) -> y
+    w4a8_mmq_workspace_size(M, N, K)
+    w4_check_device_error()
+"""
+from __future__ import annotations
+
+from ._lib import (LibraryMissing, W4_OK, W4_OUT_BF16, W4_OUT_F32, load, status_string)
+
+__all__ = [
+    "W4Error", "LibraryMissing", "w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv",
+    "q8_quantize_act", "w4a8_mmq", "w4a8_mmq_workspace_size", "w4_check_device_error",
+    "w4_abi_version", "lib",
+]
+
+GROUP = 256
+BLOCK = 32
+
+
+class W4Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = int(code)
+        msg = status_string(code)
+        if code == 6:  # W4_ERR_CUDA
+            msg += f" (cudaError {load().w4_last_cuda_error()})"
+        super().__init__(f"{what}: {msg}")
+
+
+def lib():
+    """The loaded ctypes library (raw C ABI)."""
+    return load()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _check(code: int, what: str):
+    if code != W4_OK:
+        raise W4Error(code, what)
+
+
+def _stream(stream=None) -> int:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t) -> int:
+    return t.data_ptr()
+
+
+def _need(t, dtype, name: str, ndim: int = 2):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _as_u16(t):
+    torch = _torch()
+    if t.dtype in (torch.bfloat16, torch.float16):
+        return t.view(torch.int16)
+    return t
+
+
+def w4_abi_version() -> int:
+    return int(load().w4_abi_version())
+
+
+def w4_check_device_error() -> None:
+    """Synchronise and raise if a kernel reported a timed-out wait."""
+    _check(load().w4_check_device_error(), "w4_check_device_error")
+
+
+def w4_pack(w, codes=None, d=None, m=None, stream=None):
+    """Quantise fp32 W[N,K] (K % 256 == 0) to W4-G256 planes.
+    Returns (codes uint8[N,K/2], d fp16[N,K/256], m fp16[N,K/256])."""
+    torch = _torch()
+    _need(w, torch.float32, "w")
+    N, K = w.shape
+    if codes is None:
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    if d is None:
+        d = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
+    if m is None:
+        m = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
+    _check(load().w4_pack(_ptr(w), N, K, _ptr(codes), _ptr(d), _ptr(m), _stream(stream)),
+           "w4_pack")
+    return codes, d, m
+
+
+def w4_pack_codes(q, codes=None, stream=None):
+    """One code per byte q uint8[N,K] -> packed codes uint8[N,K/2]."""
+    torch = _torch()
+    _need(q, torch.uint8, "q")
+    N, K = q.shape
+    if codes is None:
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=q.device)
+    _check(load().w4_pack_codes(_ptr(q), N, K, _ptr(codes), _stream(stream)), "w4_pack_codes")
+    return codes
+
+
+def w4_unpack(codes, K: int, q=None, stream=None):
+    """Packed codes uint8[N,K/2] -> one code per byte uint8[N,K]."""
+    torch = _torch()
+    _need(codes, torch.uint8, "codes")
+    N = codes.shape[0]
+    if codes.shape[1] * 2 != K:
+        raise ValueError("codes must have K/2 columns")
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.uint8, device=codes.device)
+    _check(load().w4_unpack(_ptr(codes), N, K, _ptr(q), _stream(stream)), "w4_unpack")
+    return q
+
+
+def _out_code(out_dtype) -> int:
+    torch = _torch()
+    if out_dtype in (torch.float32, "f32", "fp32", W4_OUT_F32):
+        return W4_OUT_F32
+    if out_dtype in (torch.bfloat16, "bf16", W4_OUT_BF16):
+        return W4_OUT_BF16
+    raise ValueError(f"unsupported out_dtype {out_dtype}")
+
+
+def w4_gemv(codes, d, m, x, out_dtype=None, y=None, stream=None):
+    """y[M,N] = x[M,K] @ dequant(W)^T for 1 <= M <= 8; x is bf16."""
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    _need(codes, torch.uint8, "codes")
+    _need(d, torch.float16, "d")
+    _need(m, torch.float16, "m")
+    _need(x, torch.bfloat16, "x")
+    N = codes.shape[0]
+    M, K = x.shape
+    oc = _out_code(out_dtype)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32 if oc == W4_OUT_F32 else torch.bfloat16,
+                        device=x.device)
+    _check(load().w4_gemv(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x), M, _ptr(y), oc,
+                          _stream(stream)), "w4_gemv")
+    return y
+
+
+def q8_quantize_act(x, qa=None, dx=None, bsum=None, stream=None):
+    """bf16 x[M,K] (K % 32 == 0) -> (qa int8[M,K], dx fp32[M,K/32], bsum int32[M,K/32])."""
+    torch = _torch()
+    _need(x, torch.bfloat16, "x")
+    M, K = x.shape
+    if qa is None:
+        qa = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if dx is None:
+        dx = torch.empty((M, K // BLOCK), dtype=torch.float32, device=x.device)
+    if bsum is None:
+        bsum = torch.empty((M, K // BLOCK), dtype=torch.int32, device=x.device)
+    _check(load().q8_quantize_act(_ptr(x), M, K, _ptr(qa), _ptr(dx), _ptr(bsum),
+                                  _stream(stream)), "q8_quantize_act")
+    return qa, dx, bsum
+
+
+def w4a8_mmq_workspace_size(M: int, N: int, K: int) -> int:
+    return int(load().w4a8_mmq_workspace_size(M, N, K))
+
+
+def w4a8_mmq(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, workspace=None, stream=None):
+    """y[M,N] from W4-G256 weights and int8 activation blocks (tensor cores)."""
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    _need(codes, torch.uint8, "codes")
+    _need(d, torch.float16, "d")
+    _need(m, torch.float16, "m")
+    _need(qa, torch.int8, "qa")
+    _need(dx, torch.float32, "dx")
+    _need(bsum, torch.int32, "bsum")
+    N = codes.shape[0]
+    M, K = qa.shape
+    oc = _out_code(out_dtype)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32 if oc == W4_OUT_F32 else torch.bfloat16,
+                        device=qa.device)
+    ws_need = w4a8_mmq_workspace_size(M, N, K)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=qa.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(load().w4a8_mmq(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(qa), _ptr(dx), _ptr(bsum),
+                           M, _ptr(y), oc, ws_ptr, ws_bytes, _stream(stream)), "w4a8_mmq")
+    return y

@@ -1,0 +1,527 @@
+// mmq.cu -- W4A8 prefill product on the sm_100a int8 tensor cores.
+//
+// The hipfire HFQ4-G256 MMQ article ("What changed" list) pre-quantises the
+// prefill activations to a Q8_1-style int8 block layout and runs a tiled int8
+// matrix-matrix product over the 4-bit weights, applying the scales after the
+// integer products.  Here:
+//
+//   P[t][n][b] = sum_{k in block b} q[n][k] * qa[t][k]          (exact int32)
+//   y[t][n]    = sum_g ( d[n][g] * sum_{b in g} dx[t][b] * P[t][n][b]
+//                        + m[n][g] * sum_{b in g} dx[t][b] * S[t][b] )
+//
+// One CTA computes a 128 (tokens) x 128 (weight rows) tile of y, looping over
+// K in stages of 128 (four 32-element activation blocks):
+//   warp 0      TMA producer: the qa tile (128 x 128 B, 128B-swizzled) and the
+//               packed code tile (128 rows x 64 B) into a 4-stage ring.
+//   warp 1      allocates 512 TMEM columns; one lane issues, per 32-block, one
+//               tcgen05.mma.kind::i8 (M=128, N=128, K=32; A = qa as s8, B = the
+//               codes as u8) into its own 128-column TMEM buffer, overwriting
+//               it, so every block's exact int32 products stay separate.
+//   warps 2-3   unpack each code tile, nibble -> byte, into the 128B-swizzled
+//               K-major layout the MMA's shared-memory descriptor expects
+//               (tcgen05 has no 4-bit integer kind).
+//   warps 4-11  epilogue: each thread owns one token row (its TMEM lane) and 64
+//               weight rows; per block it loads the 64 int32 products, releases
+//               the buffer, and accumulates dx[t][b] * P into a per-group sum;
+//               at each group end it applies d[n][g] and the exact min term
+//               m[n][g] * sum_b dx[t][b] S[t][b].
+// The MMA runs up to four blocks ahead of the epilogue (four TMEM buffers).
+// Registers are rebalanced with setmaxnreg: 72 per thread for warps 0-3, 216
+// for the epilogue (128*72 + 256*216 = 384*168, the launch allotment).
+// Every mbarrier wait is bounded; a wait that runs out raises the CTA's abort
+// flag and the device error word, all roles drain what they issued, TMEM is
+// freed and the CTA returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int BM = 128;        // tokens per tile (MMA M, TMEM lanes)
+constexpr int BN = 128;        // weight rows per tile (MMA N)
+constexpr int BK = 128;        // K elements per pipeline stage
+constexpr int KB = 32;         // activation block = MMA K for kind::i8
+constexpr int STAGES = 4;
+constexpr int NBUF = BK / KB;  // TMEM buffers, one per block of a stage
+constexpr int kThreads = 384;
+constexpr int A_BYTES = BM * BK;
+constexpr int B_BYTES = BN * BK;
+constexpr int BP_BYTES = BN * BK / 2;
+constexpr int TMEM_COLS = NBUF * BN;  // 512
+constexpr int kMaxGroups = 64;        // K <= 16384
+
+static_assert(TMEM_COLS == 512, "TMEM allocation must be a power of two <= 512");
+
+struct Smem {
+    static constexpr int a = 0;
+    static constexpr int b = a + STAGES * A_BYTES;
+    static constexpr int bp = b + STAGES * B_BYTES;
+    static constexpr int bars = bp + STAGES * BP_BYTES;  // uint64 barriers
+    static constexpr int nbars = 3 * STAGES + 2 * NBUF + 1;
+    static constexpr int misc = bars + nbars * 8;        // tmem base, abort flag
+    static constexpr int dm = (misc + 16 + 15) & ~15;    // fp32 d[G][BN], m[G][BN]
+    static size_t total(int G) { return (size_t)dm + (size_t)2 * G * BN * 4 + 1024; }
+};
+
+struct Params {
+    const __half* d;
+    const __half* m;
+    const float* dx;
+    const int32_t* S;
+    void* y;
+    int M, N, K;
+    int out_f32;
+    int* err;
+};
+
+// ---------------------------------------------------------------------------
+// tcgen05 wrappers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    // K-major, 128-byte swizzle: 8-row core groups 1024 bytes apart.
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            w4::smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// kernel
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(kThreads, 1)
+    w4a8_mmq_kernel(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b, const Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte alignment of the operand tiles (128B swizzle atoms).
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sa = smem + Smem::a;
+    uint8_t* sb = smem + Smem::b;
+    uint8_t* sbp = smem + Smem::bp;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bars);
+    uint64_t* full = bars;                   // TMA landed (A + packed B)
+    uint64_t* unpacked = bars + STAGES;      // B unpacked into the MMA layout
+    uint64_t* empty = bars + 2 * STAGES;     // MMAs of the stage done
+    uint64_t* tfull = bars + 3 * STAGES;     // TMEM buffer written
+    uint64_t* tempty = tfull + NBUF;         // TMEM buffer drained
+    uint64_t* drain = tempty + NBUF;         // final MMA completion
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Smem::misc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
+    float* d_s = reinterpret_cast<float*>(smem + Smem::dm);
+    const int G = p.K / 256;
+    float* m_s = d_s + G * BN;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN;
+    const int m0 = blockIdx.y * BM;
+    const int ksteps = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            w4::mbar_init(&full[i], 1);
+            w4::mbar_init(&unpacked[i], 2);
+            w4::mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < NBUF; ++i) {
+            w4::mbar_init(&tfull[i], 1);
+            w4::mbar_init(&tempty[i], 8);
+        }
+        w4::mbar_init(drain, 1);
+        *abort_flag = 0;
+        w4::fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         w4::smem_u32((const void*)tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    // epilogue threads stage this tile's d and m (fp32, [g][n]); rows past N -> 0
+    if (warp >= 4) {
+        const int e = threadIdx.x - 128;
+        for (int i = e; i < BN * G; i += 256) {
+            const int r = i / G, g = i - r * G;
+            const int n = n0 + r;
+            float dv = 0.0f, mv = 0.0f;
+            if (n < p.N) {
+                dv = __half2float(p.d[(size_t)n * G + g]);
+                mv = __half2float(p.m[(size_t)n * G + g]);
+            }
+            d_s[g * BN + r] = dv;
+            m_s[g * BN + r] = mv;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+        if (warp == 0) {
+            // ---------------- TMA producer ----------------
+            if (w4::elect_one()) {
+                w4::prefetch_tmap(&tm_a);
+                w4::prefetch_tmap(&tm_b);
+                int issued = 0;
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int s = ks % STAGES;
+                    const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
+                    if (!w4::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err)) break;
+                    w4::mbar_arrive_expect_tx(&full[s], A_BYTES + BP_BYTES);
+                    w4::tma_load_2d(sa + s * A_BYTES, &tm_a, &full[s], ks * BK, m0);
+                    w4::tma_load_2d(sbp + s * BP_BYTES, &tm_b, &full[s], ks * (BK / 2), n0);
+                    issued = ks + 1;
+                }
+                // drain: every issued load must land before the CTA exits
+                for (int ks = issued - STAGES < 0 ? 0 : issued - STAGES; ks < issued; ++ks)
+                    w4::mbar_wait(&full[ks % STAGES], (uint32_t)(ks / STAGES) & 1u, nullptr,
+                                  p.err);
+            }
+        } else if (warp == 1) {
+            // ---------------- MMA issuer ----------------
+            if (w4::elect_one()) {
+                constexpr uint32_t idesc = (2u << 4)             // D: s32
+                                           | (1u << 7)           // A: s8
+                                           | (0u << 10)          // B: u8
+                                           | ((uint32_t)(BN >> 3) << 17)
+                                           | ((uint32_t)(BM >> 4) << 24);
+                for (int ks = 0; ks < ksteps; ++ks) {
+                    const int s = ks % STAGES;
+                    const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
+                    if (!w4::mbar_wait(&full[s], ph, abort_flag, p.err)) break;
+                    if (!w4::mbar_wait(&unpacked[s], ph, abort_flag, p.err)) break;
+                    tc_fence_after();
+                    const uint32_t a_addr = w4::smem_u32(sa + s * A_BYTES);
+                    const uint32_t b_addr = w4::smem_u32(sb + s * B_BYTES);
+                    bool ok = true;
+                    for (int q = 0; q < NBUF; ++q) {
+                        if (!w4::mbar_wait(&tempty[q], ((uint32_t)ks & 1u) ^ 1u, abort_flag,
+                                           p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        mma_i8(tmem_base + (uint32_t)(q * BN), smem_desc_sw128(a_addr + q * KB),
+                               smem_desc_sw128(b_addr + q * KB), idesc, 0u);
+                        mma_commit(&tfull[q]);
+                    }
+                    mma_commit(&empty[s]);
+                    if (!ok) break;
+                }
+                mma_commit(drain);
+                w4::mbar_wait(drain, 0u, nullptr, p.err);
+            }
+        } else {
+            // ---------------- unpackers (warps 2, 3) ----------------
+            const int ut = threadIdx.x - 64;  // 0..63
+            for (int ks = 0; ks < ksteps; ++ks) {
+                const int s = ks % STAGES;
+                const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
+                if (!w4::mbar_wait(&full[s], ph, abort_flag, p.err)) break;
+                const uint8_t* src = sbp + s * BP_BYTES;
+                uint8_t* dst = sb + s * B_BYTES;
+#pragma unroll 4
+                for (int it = 0; it < (BN * 8) / 64; ++it) {
+                    const int item = it * 64 + ut;
+                    const int r = item >> 3, jc = item & 7;  // row, 16-code chunk
+                    const uint2 pk = *reinterpret_cast<const uint2*>(src + r * (BK / 2) + jc * 8);
+                    const uint32_t lo0 = pk.x & 0x0F0F0F0Fu, hi0 = (pk.x >> 4) & 0x0F0F0F0Fu;
+                    const uint32_t lo1 = pk.y & 0x0F0F0F0Fu, hi1 = (pk.y >> 4) & 0x0F0F0F0Fu;
+                    uint4 o;
+                    o.x = __byte_perm(lo0, hi0, 0x5140);
+                    o.y = __byte_perm(lo0, hi0, 0x7362);
+                    o.z = __byte_perm(lo1, hi1, 0x5140);
+                    o.w = __byte_perm(lo1, hi1, 0x7362);
+                    *reinterpret_cast<uint4*>(dst + r * BK + ((jc ^ (r & 7)) << 4)) = o;
+                }
+                w4::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) w4::mbar_arrive(&unpacked[s]);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 4..11) ----------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+        const int quarter = warp & 3;               // TMEM lane quarter of this warp
+        const int h = (warp - 4) >> 2;              // column half: 64 weight rows
+        const int row = quarter * 32 + lane;        // token row within the tile
+        const int t = m0 + row;
+        const bool t_live = t < p.M;
+        const int B = p.K / KB;
+        const uint32_t tm_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(h * 64);
+        float acc[64], yv[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+            acc[c] = 0.0f;
+            yv[c] = 0.0f;
+        }
+        float dxg[8];
+        float tmin = 0.0f;
+        bool ok = true;
+        for (int ks = 0; ks < ksteps && ok; ++ks) {
+#pragma unroll 1
+            for (int q = 0; q < NBUF; ++q) {
+                const int kb = ks * NBUF + q;
+                const int g = kb >> 3;
+                if ((kb & 7) == 0) {
+                    // activation scales and block sums of this group (32-byte aligned)
+                    if (t_live) {
+                        const float4* dp = reinterpret_cast<const float4*>(p.dx + (size_t)t * B + g * 8);
+                        const int4* sp = reinterpret_cast<const int4*>(p.S + (size_t)t * B + g * 8);
+                        const float4 a0 = __ldg(dp), a1 = __ldg(dp + 1);
+                        const int4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
+                        dxg[0] = a0.x; dxg[1] = a0.y; dxg[2] = a0.z; dxg[3] = a0.w;
+                        dxg[4] = a1.x; dxg[5] = a1.y; dxg[6] = a1.z; dxg[7] = a1.w;
+                        tmin = dxg[0] * (float)s0.x;
+                        tmin = fmaf(dxg[1], (float)s0.y, tmin);
+                        tmin = fmaf(dxg[2], (float)s0.z, tmin);
+                        tmin = fmaf(dxg[3], (float)s0.w, tmin);
+                        tmin = fmaf(dxg[4], (float)s1.x, tmin);
+                        tmin = fmaf(dxg[5], (float)s1.y, tmin);
+                        tmin = fmaf(dxg[6], (float)s1.z, tmin);
+                        tmin = fmaf(dxg[7], (float)s1.w, tmin);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) dxg[i] = 0.0f;
+                        tmin = 0.0f;
+                    }
+                }
+                if (!w4::mbar_wait(&tfull[q], (uint32_t)ks & 1u, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tm_row + (uint32_t)(q * BN), r0);
+                tmem_ld32(tm_row + (uint32_t)(q * BN + 32), r1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) w4::mbar_arrive(&tempty[q]);
+                float dxb = dxg[0];
+#pragma unroll
+                for (int i = 1; i < 8; ++i)
+                    if ((kb & 7) == i) dxb = dxg[i];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    acc[c] = fmaf(dxb, (float)(int)r0[c], acc[c]);
+                    acc[32 + c] = fmaf(dxb, (float)(int)r1[c], acc[32 + c]);
+                }
+                if ((kb & 7) == 7) {
+                    const float4* dg = reinterpret_cast<const float4*>(d_s + g * BN + h * 64);
+                    const float4* mg = reinterpret_cast<const float4*>(m_s + g * BN + h * 64);
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        const float4 dv = dg[c4], mv = mg[c4];
+                        yv[4 * c4 + 0] = fmaf(dv.x, acc[4 * c4 + 0], fmaf(mv.x, tmin, yv[4 * c4 + 0]));
+                        yv[4 * c4 + 1] = fmaf(dv.y, acc[4 * c4 + 1], fmaf(mv.y, tmin, yv[4 * c4 + 1]));
+                        yv[4 * c4 + 2] = fmaf(dv.z, acc[4 * c4 + 2], fmaf(mv.z, tmin, yv[4 * c4 + 2]));
+                        yv[4 * c4 + 3] = fmaf(dv.w, acc[4 * c4 + 3], fmaf(mv.w, tmin, yv[4 * c4 + 3]));
+                        acc[4 * c4 + 0] = 0.0f;
+                        acc[4 * c4 + 1] = 0.0f;
+                        acc[4 * c4 + 2] = 0.0f;
+                        acc[4 * c4 + 3] = 0.0f;
+                    }
+                }
+            }
+        }
+        if (ok && t_live) {
+            const int nb = n0 + h * 64;
+            if (p.out_f32) {
+                float* yr = reinterpret_cast<float*>(p.y) + (size_t)t * p.N;
+                if (nb + 64 <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4)
+                        *reinterpret_cast<float4*>(yr + nb + 4 * c4) =
+                            make_float4(yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (nb + c < p.N) yr[nb + c] = yv[c];
+                }
+            } else {
+                __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)t * p.N;
+                if (nb + 64 <= p.N && (p.N & 7) == 0) {
+#pragma unroll
+                    for (int c8 = 0; c8 < 8; ++c8) {
+                        uint4 v;
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(yv[8 * c8 + 0], yv[8 * c8 + 1]);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(yv[8 * c8 + 2], yv[8 * c8 + 3]);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(yv[8 * c8 + 4], yv[8 * c8 + 5]);
+                        __nv_bfloat162 h3 = __floats2bfloat162_rn(yv[8 * c8 + 6], yv[8 * c8 + 7]);
+                        v.x = *reinterpret_cast<uint32_t*>(&h0);
+                        v.y = *reinterpret_cast<uint32_t*>(&h1);
+                        v.z = *reinterpret_cast<uint32_t*>(&h2);
+                        v.w = *reinterpret_cast<uint32_t*>(&h3);
+                        *reinterpret_cast<uint4*>(yr + nb + 8 * c8) = v;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (nb + c < p.N) yr[nb + c] = __float2bfloat16_rn(yv[c]);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host: tensor maps
+// ---------------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+// 2-D uint8 tensor map over a dense row-major [rows][cols] byte matrix.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                 uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K) {
+    (void)M;
+    (void)N;
+    (void)K;
+    return 0;
+}
+
+int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
+             int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
+             void* y, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
+    if (K / 256 > kMaxGroups || M > (1 << 24) || N > (1 << 24)) return W4_ERR_SHAPE;
+    if (out_dtype != W4_OUT_BF16 && out_dtype != W4_OUT_F32) return W4_ERR_SHAPE;
+    if (!codes || !d_f16 || !m_f16 || !qa || !dx || !bsum || !y) return W4_ERR_NULL;
+    if (!w4::aligned16(codes) || !w4::aligned16(d_f16) || !w4::aligned16(m_f16) ||
+        !w4::aligned16(qa) || !w4::aligned16(dx) || !w4::aligned16(bsum) || !w4::aligned16(y))
+        return W4_ERR_ALIGN;
+    int rc = w4::check_device();
+    if (rc != W4_OK) return rc;
+    int* err = w4::device_error_word();
+    if (!err) return W4_ERR_CUDA;
+
+    CUtensorMap ma, mb;
+    if (!make_map_u8(&ma, qa, (uint64_t)K, (uint64_t)M, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+        return W4_ERR_CUDA;
+    if (!make_map_u8(&mb, codes, (uint64_t)K / 2, (uint64_t)N, BK / 2, BN,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+        return W4_ERR_CUDA;
+
+    const int G = (int)(K / 256);
+    const size_t smem = Smem::total(G);
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return w4::cuda_fail(e);
+    if (attr_dev != dev) {
+        e = cudaFuncSetAttribute(w4a8_mmq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)Smem::total(kMaxGroups));
+        if (e != cudaSuccess) return w4::cuda_fail(e);
+        attr_dev = dev;
+    }
+    Params prm;
+    prm.d = reinterpret_cast<const __half*>(d_f16);
+    prm.m = reinterpret_cast<const __half*>(m_f16);
+    prm.dx = dx;
+    prm.S = bsum;
+    prm.y = y;
+    prm.M = (int)M;
+    prm.N = (int)N;
+    prm.K = (int)K;
+    prm.out_f32 = out_dtype == W4_OUT_F32;
+    prm.err = err;
+    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    w4a8_mmq_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, prm);
+    return w4::launch_status();
+}
+
+}  // extern "C"

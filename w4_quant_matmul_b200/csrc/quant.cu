@@ -1,0 +1,84 @@
+// quant.cu -- activation quantiser to int8 blocks of 32 (the Q8_1-style MMQ
+// layout the hipfire prefill path pre-quantises activations to: "What
+// changed" list of the hipfire HFQ4-G256 MMQ article).
+//
+// Per (token t, block b of 32 consecutive k):
+//   amax = max |x|;  dx = amax / 127 (IEEE fp32 division);
+//   amax == 0 -> dx = 0, qa = 0, S = 0;
+//   else qa = clamp(rint(x / dx), -127, 127) (ties to even);  S = sum(qa).
+//
+// HBM-bound: 2 bytes read and 1.25 bytes written per element.  Each thread
+// owns 8 consecutive elements (one 16-byte load); four adjacent lanes form a
+// block and reduce amax and S with two xor-shuffles.  K % 32 == 0 means a
+// block never straddles a row, so the flattened [M][K] array is processed as
+// one stream.
+#include "common.cuh"
+
+namespace {
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __restrict__ x,
+                                                          int64_t n8, int8_t* __restrict__ qa,
+                                                          float* __restrict__ dx,
+                                                          int32_t* __restrict__ bsum) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    // n8 (number of 8-element chunks) is a multiple of 4, so every warp-wide
+    // iteration is either all live or all dead within each group of 4 lanes;
+    // the loop bound keeps whole warps together for the shuffles.
+    const int64_t n8_warp = (n8 + 31) & ~int64_t(31);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8_warp; i += stride) {
+        const bool live = i < n8;
+        uint4 v = live ? __ldg(reinterpret_cast<const uint4*>(x) + i) : make_uint4(0, 0, 0, 0);
+        float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                      bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+        float amax = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const float scale = __fdiv_rn(amax, 127.0f);
+        int sum = 0;
+        uint32_t packed[2] = {0u, 0u};
+        if (amax != 0.0f) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float qf = rintf(__fdiv_rn(f[j], scale));
+                qf = fminf(fmaxf(qf, -127.0f), 127.0f);
+                const int qi = (int)qf;
+                sum += qi;
+                packed[j >> 2] |= ((uint32_t)qi & 0xFFu) << (8 * (j & 3));
+            }
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+        if (live) {
+            reinterpret_cast<uint2*>(qa)[i] = make_uint2(packed[0], packed[1]);
+            if ((i & 3) == 0) {
+                dx[i >> 2] = (amax == 0.0f) ? 0.0f : scale;
+                bsum[i >> 2] = sum;
+            }
+        }
+    }
+}
+
+}  // namespace
+
+extern "C" int q8_quantize_act(const uint16_t* x_bf16, int64_t M, int64_t K, int8_t* qa,
+                               float* dx, int32_t* bsum, void* stream) {
+    if (M < 0 || K < 0 || K % 32 != 0) return W4_ERR_SHAPE;
+    if (M == 0 || K == 0) return W4_OK;
+    if (!x_bf16 || !qa || !dx || !bsum) return W4_ERR_NULL;
+    if (!w4::aligned16(x_bf16) || !w4::aligned16(qa) || !w4::aligned16(dx) ||
+        !w4::aligned16(bsum))
+        return W4_ERR_ALIGN;
+    int rc = w4::check_device();
+    if (rc != W4_OK) return rc;
+    const int64_t n8 = M * K / 8;
+    int64_t blocks = (n8 + 255) / 256;
+    const int64_t cap = (int64_t)w4::sm_count() * 16;
+    if (blocks > cap) blocks = cap;
+    q8_quantize_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(x_bf16, n8, qa, dx, bsum);
+    return w4::launch_status();
+}
