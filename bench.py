@@ -238,41 +238,58 @@ class Workload:
         return self.x[M], self.y[M]
 
 
-def time_gemv_sweep(torch, w4, wl, M, steps, warmup, stream, dom_index=4):
-    """Times `steps` sweeps; returns (elapsed_s, per-shape mean ms, launches)."""
+def _capture(torch, stream, fn):
+    """Capture fn() (launches on `stream`) into a CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()  # eager once: per-kernel attributes and caches set outside capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_gemv_sweep(torch, w4, wl, M, steps, warmup, stream):
+    """Times `steps` sweeps of the five GEMVs, each step one CUDA-graph replay
+    (the two weight copies alternate).  Returns (elapsed_s, per-shape mean ms,
+    kernel launches in the timed region)."""
     xs, ys = wl.xs(M)
     ncopy = len(wl.weights)
 
-    def step(i, ev=None):
-        wset = wl.weights[i % ncopy]
-        for s in range(len(SHAPES)):
-            codes, d, m = wset[s]
-            if ev is not None:
-                ev[s][0].record(stream)
-            w4.w4_gemv(codes, d, m, xs[s], out_dtype=torch.bfloat16, y=ys[s], stream=stream)
-            if ev is not None:
-                ev[s][1].record(stream)
+    def gemv(c, s):
+        codes, d, m = wl.weights[c][s]
+        w4.w4_gemv(codes, d, m, xs[s], out_dtype=torch.bfloat16, y=ys[s], stream=stream)
 
-    for i in range(warmup):
-        step(i)
-    torch.cuda.synchronize()
-    # pass 1: the whole timed region, bracketed by events only
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(steps):
-        step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    elapsed = start.elapsed_time(end) / 1e3
-    # pass 2: per-launch events on the launching stream (per-kernel times)
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in SHAPES]
-           for _ in range(steps)]
-    for i in range(steps):
-        step(i, evs[i])
-    torch.cuda.synchronize()
+    steps_g = [_capture(torch, stream, lambda c=c: [gemv(c, s) for s in range(len(SHAPES))])
+               for c in range(ncopy)]
+    shape_g = [[_capture(torch, stream, lambda c=c, s=s: gemv(c, s)) for s in range(len(SHAPES))]
+               for c in range(ncopy)]
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            steps_g[i % ncopy].replay()
+        torch.cuda.synchronize()
+        # the timed region: K steps bracketed by events on the launching stream
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(steps):
+            steps_g[i % ncopy].replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        elapsed = start.elapsed_time(end) / 1e3
+        # per-kernel durations: one graph per launch, events between them
+        evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in SHAPES]
+               for _ in range(steps)]
+        for i in range(steps):
+            for s in range(len(SHAPES)):
+                evs[i][s][0].record(stream)
+                shape_g[i % ncopy][s].replay()
+                evs[i][s][1].record(stream)
+        torch.cuda.synchronize()
     per = [statistics.mean(evs[i][s][0].elapsed_time(evs[i][s][1]) for i in range(steps))
            for s in range(len(SHAPES))]
+    del steps_g, shape_g
     return elapsed, per, steps * len(SHAPES)
 
 
@@ -494,7 +511,8 @@ def run_ours(args):
                                    "(151936,2560), M=1, bf16 out",
                        "global_batch": world, "seq_len": 1,
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2: two 253 MB weight sets alternate"},
+                       "l2": "inputs larger than L2: two 253 MB weight sets alternate",
+                       "launch": "each step replays a CUDA graph of the five GEMVs"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk.summary(), "cpu_baseline": cpu,
         }
@@ -578,6 +596,39 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """One kernel configuration launched `--reps` times on device-resident
+    synthetic inputs (the command the committed ncu summaries capture)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    import w4_quant_matmul_b200 as w4
+    g = torch.Generator(device=dev)
+    g.manual_seed(17)
+    N, K, M = args.N, args.K, args.M
+    w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
+    codes, d, m = w4.w4_pack(w)
+    del w
+    torch.cuda.synchronize()
+    x = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+    if args.case == "gemv":
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(args.reps):
+            w4.w4_gemv(codes, d, m, x, out_dtype=torch.bfloat16, y=y)
+    elif args.case == "quant":
+        qa, dx, S = w4.q8_quantize_act(x)
+        for _ in range(args.reps):
+            w4.q8_quantize_act(x, qa, dx, S)
+    else:
+        qa, dx, S = w4.q8_quantize_act(x)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(args.reps):
+            w4.w4a8_mmq(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y)
+    torch.cuda.synchronize()
+    w4.w4_check_device_error()
+    print(json.dumps({"case": args.case, "N": N, "K": K, "M": M, "reps": args.reps, "ok": True}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -587,10 +638,18 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="only the timed batch-1 sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--case", choices=["gemv", "mmq", "quant"],
+                    help="launch one kernel configuration --reps times (profiling)")
+    ap.add_argument("--N", type=int, default=151936)
+    ap.add_argument("--K", type=int, default=2560)
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--reps", type=int, default=5)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.case:
+        run_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -5,25 +5,35 @@
 //   y[t][n] = sum_g ( d[n][g] * sum_{k in g} q[n][k] x[t][k]
 //                     + m[n][g] * sum_{k in g} x[t][k] )
 //
-// Design (HBM-bound: 0.515625 bytes of weight per multiply-add at M = 1):
-//  * A half-warp (16 lanes) owns RH whole rows; lane j streams 16-byte code
-//    chunks (32 codes) c = j, j+16, ... of each row with non-allocating
-//    128-bit loads, U chunks ahead, so every lane keeps U*RH loads in flight.
-//    No cross-warp reduction: a 4-step xor-shuffle inside the half-warp
-//    finishes each row.
-//  * The activations are staged once per CTA into shared memory as fp32 in
-//    a chunk-minor layout (sub-block i of chunk c at [i][c]) so that the 16
-//    lanes, which read 16 different chunks, hit 16 different banks; the
-//    per-chunk sums Sx[t][c] are staged beside them.  When M*K*4 bytes do not
-//    fit, x stays bf16 in shared memory and is widened on use.
-//  * Dequantisation never materialises w: a code q becomes the float
-//    1 + q/16 by placing its nibble in the top mantissa bits of 1.0f (one
-//    shift and one logic op), so per chunk
-//      A = sum x * (1 + q/16)   and   sum q*x = 16 * (A - Sx),
-//    and the group's contribution is 16 d (A - Sx) + m Sx, applied once per
-//    chunk.  Accumulation is fp32 in a fixed order (bitwise deterministic).
-//  * Persistent grid: CTAs loop over blocks of 16*RH rows, so the activation
-//    staging is paid once per CTA.
+// HBM-bound at M = 1 (0.515625 weight bytes per multiply-add), so the design
+// goal is a weight stream that keeps enough bytes in flight and an inner loop
+// cheap enough not to become the limit:
+//
+//  * Work split.  A half-warp (16 lanes) owns RH rows and one of KS K-slices;
+//    lane j streams the 16-byte code chunks (32 codes) c = j, j+16, ... of its
+//    slice with non-allocating 128-bit loads, U chunks ahead per row.  With
+//    KS > 1 the slices of a row are summed in fixed order through shared
+//    memory (small-N shapes need the extra streams); with KS = 1 a 4-step
+//    xor-shuffle finishes the row.  CTAs loop over row blocks.
+//  * Dequantisation.  Two codes at a time become a bf16x2 pair (128 + q) by
+//    OR-ing their nibbles, shifted to bits 0-3 of each half, into the bf16
+//    exponent of 128: one logic op for k and k+4 of a word, a shift and a logic
+//    op for the other three pairs.  The mixed-precision fma.rn.f32.bf16 then
+//    accumulates x * (128 + q) in fp32 at full FMA rate, exactly (8-bit x 8-bit
+//    products), so per 32-code chunk
+//        A = sum x (128 + q)   and   sum q x = A - 128 * Sx,
+//    and the chunk adds d (A - 128 Sx) + m Sx (Sx = sum of its 32 x).
+//  * Activations.  x is staged once per CTA into shared memory as bf16 pairs
+//    permuted to match the code pairs, chunk-minor (sub-word w of chunk c at
+//    [w][c]) so the 16 lanes of a half-warp hit 16 different banks; the chunk
+//    sums Sx are staged beside them (fp32, fixed order).
+//  * Programmatic dependent launch.  Before griddepcontrol.wait the CTA only
+//    asks L2 to prefetch its first batch of weights (bulk L2 prefetch; L2 is
+//    the point of coherence, so a prefetch can never observe stale data even
+//    if the preceding kernel writes the weights).  In a chain of launches the
+//    first HBM round trip of this GEMV overlaps the tail of the previous
+//    kernel; every load that feeds arithmetic happens after the wait.
+// Accumulation is fp32 in a fixed order: results are bitwise deterministic.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -43,170 +53,206 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     return r;
 }
 
-__device__ __forceinline__ float ld_f16_as_f32(const __half* p) { return __half2float(__ldg(p)); }
-
-// 1 + q/16 for the nibble at bit position 4*i of w.
-template <int I>
-__device__ __forceinline__ float nib_f(uint32_t w) {
-    constexpr int s = 19 - 4 * I;
-    const uint32_t v = (s >= 0) ? (w << (s >= 0 ? s : 0)) : (w >> (s < 0 ? -s : 0));
-    return __uint_as_float((v & 0x00780000u) | 0x3F800000u);
+__device__ __forceinline__ uint16_t ld_nc_u16(const void* p) {
+    uint16_t r;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));
+    return r;
 }
 
-template <int M, bool XF32>
-struct XStage {
-    // fp32: float4 xs[M][8][C] ; bf16: uint4 xs[M][4][C]
-    static constexpr int kVecPerChunk = XF32 ? 8 : 4;
+// acc += lo(xp) * lo(fp) + hi(xp) * hi(fp), each product exact, fp32 accumulate.
+__device__ __forceinline__ float fma_bf16x2(uint32_t xp, uint32_t fp, float acc) {
+    asm("{\n\t.reg .b16 xl, xh, fl, fh;\n\t"
+        "mov.b32 {xl, xh}, %1;\n\t"
+        "mov.b32 {fl, fh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, xl, fl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, xh, fh, %0;\n\t}\n"
+        : "+f"(acc)
+        : "r"(xp), "r"(fp));
+    return acc;
+}
+
+// bf16x2 (128 + q_lo, 128 + q_hi) from the nibbles at bits [s, s+4) and
+// [s+16, s+20) of a code word.
+template <int S>
+__device__ __forceinline__ uint32_t code_pair(uint32_t w) {
+    return ((w >> S) & 0x000F000Fu) | 0x43004300u;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void l2_prefetch(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <int RH, int U>
+struct Batch {
+    uint4 wq[U][RH];
+    uint16_t dv[U][RH], mv[U][RH];
 };
 
-template <int M, int RH, int U, bool XF32>
+template <int RH, int U>
+__device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __restrict__ codes,
+                                           const __half* __restrict__ d,
+                                           const __half* __restrict__ m, const int (&rows)[RH],
+                                           size_t row_bytes, int G, int c0, int c_end) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int c = c0 + 16 * u;
+        const bool live = c < c_end;
+        const int g = (live ? c : 0) >> 3;
+#pragma unroll
+        for (int i = 0; i < RH; ++i) {
+            if (live) {
+                b.wq[u][i] = ld_nc_v4(codes + rows[i] * row_bytes + (size_t)c * 16);
+                b.dv[u][i] = ld_nc_u16(d + (size_t)rows[i] * G + g);
+                b.mv[u][i] = ld_nc_u16(m + (size_t)rows[i] * G + g);
+            } else {
+                b.wq[u][i] = make_uint4(0, 0, 0, 0);
+                b.dv[u][i] = 0;
+                b.mv[u][i] = 0;
+            }
+        }
+    }
+}
+
+template <int M, int RH, int U>
+__device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4* __restrict__ xs,
+                                              const float* __restrict__ sx, int C, int c0,
+                                              int c_end, float (&yacc)[M][RH]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int c = c0 + 16 * u;
+        if (c >= c_end) break;
+        float a[M][RH];
+#pragma unroll
+        for (int t = 0; t < M; ++t)
+#pragma unroll
+            for (int i = 0; i < RH; ++i) a[t][i] = 0.0f;
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+            uint4 xv[M];
+#pragma unroll
+            for (int t = 0; t < M; ++t) xv[t] = xs[((size_t)t * 4 + wi) * C + c];
+#pragma unroll
+            for (int i = 0; i < RH; ++i) {
+                const uint32_t w = wi == 0 ? b.wq[u][i].x
+                                 : wi == 1 ? b.wq[u][i].y
+                                 : wi == 2 ? b.wq[u][i].z
+                                           : b.wq[u][i].w;
+                const uint32_t f0 = code_pair<0>(w), f1 = code_pair<4>(w);
+                const uint32_t f2 = code_pair<8>(w), f3 = code_pair<12>(w);
+#pragma unroll
+                for (int t = 0; t < M; ++t) {
+                    a[t][i] = fma_bf16x2(xv[t].x, f0, a[t][i]);
+                    a[t][i] = fma_bf16x2(xv[t].y, f1, a[t][i]);
+                    a[t][i] = fma_bf16x2(xv[t].z, f2, a[t][i]);
+                    a[t][i] = fma_bf16x2(xv[t].w, f3, a[t][i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < M; ++t) {
+            const float s = sx[t * C + c];
+#pragma unroll
+            for (int i = 0; i < RH; ++i) {
+                const float dd = __half2float(__ushort_as_half(b.dv[u][i]));
+                const float mm = __half2float(__ushort_as_half(b.mv[u][i]));
+                yacc[t][i] = fmaf(dd, fmaf(-128.0f, s, a[t][i]), fmaf(mm, s, yacc[t][i]));
+            }
+        }
+    }
+}
+
+template <int M, int RH, int U>
 __global__ void __launch_bounds__(kThreads) w4_gemv_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
-    int N, int K, const uint16_t* __restrict__ x, void* __restrict__ y, int out_f32) {
+    int N, int K, int KS, const uint16_t* __restrict__ x, void* __restrict__ y, int out_f32) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int C = K >> 5;  // 32-code chunks per row
     const int G = K >> 8;  // groups per row
-    constexpr int VPC = XStage<M, XF32>::kVecPerChunk;
-    uint4* xs = reinterpret_cast<uint4*>(smem);                       // [M][VPC][C]
-    float* sx = reinterpret_cast<float*>(smem + (size_t)M * VPC * C * 16);  // [M][C]
+    uint4* xs = reinterpret_cast<uint4*>(smem);                                // [M][4][C]
+    float* sx = reinterpret_cast<float*>(smem + (size_t)M * 4 * C * 16);         // [M][C]
+    float* red = sx + (size_t)M * C;  // [KS][rows_per_cta][M] partial sums (KS > 1)
 
-    // ---- stage x (and the per-chunk sums) once per CTA ----
+    const int hw = threadIdx.x >> 4;  // half-warp in CTA
+    const int j = threadIdx.x & 15;   // lane in half-warp
+    const int groups = kHalfWarps / KS;  // row groups per CTA
+    const int rg = hw / KS, s = hw - (hw / KS) * KS;
+    const bool active = rg < groups;
+    const int rows_per_cta = groups * RH;
+    const int nblocks = (N + rows_per_cta - 1) / rows_per_cta;
+    const size_t row_bytes = (size_t)(K >> 1);
+    const int cs = (int)(((long long)C * s) / KS), ce = (int)(((long long)C * (s + 1)) / KS);
+
+    // ---- first batch of this CTA's weights: independent of earlier kernels ----
+    int blk = blockIdx.x;
+    int rows[RH];
+#pragma unroll
+    for (int i = 0; i < RH; ++i) {
+        const int n = blk * rows_per_cta + (active ? rg : 0) * RH + i;
+        rows[i] = n < N ? n : N - 1;  // tail rows re-read row N-1; results dropped
+    }
+    if (blk < nblocks && active && j == 0) {
+        const int c_last = min(cs + 16 * U, ce);
+        if (c_last > cs) {
+#pragma unroll
+            for (int i = 0; i < RH; ++i)
+                l2_prefetch(codes + rows[i] * row_bytes + (size_t)cs * 16,
+                            (uint32_t)(c_last - cs) * 16u);
+        }
+    }
+
+    // ---- everything below may depend on the previous kernel in the stream ----
+    pdl_wait();
+    Batch<RH, U> bt;
+    if (blk < nblocks && active) load_batch(bt, codes, d, m, rows, row_bytes, G, cs + j, ce);
+
+    // ---- x and its chunk sums, once per CTA ----
     const int nvec = M * C * 4;  // uint4 (8 bf16) units of x
     for (int v = threadIdx.x; v < nvec; v += kThreads) {
         const int t = v / (C * 4);
         const int r = v - t * C * 4;
-        const int c = r >> 2, q4 = r & 3;  // chunk, quarter (8 values)
+        const int c = r >> 2, wi = r & 3;
         const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x) + v);
-        if (XF32) {
-            float4 a, b;
-            a.x = __uint_as_float(raw.x << 16); a.y = __uint_as_float(raw.x & 0xFFFF0000u);
-            a.z = __uint_as_float(raw.y << 16); a.w = __uint_as_float(raw.y & 0xFFFF0000u);
-            b.x = __uint_as_float(raw.z << 16); b.y = __uint_as_float(raw.z & 0xFFFF0000u);
-            b.z = __uint_as_float(raw.w << 16); b.w = __uint_as_float(raw.w & 0xFFFF0000u);
-            float4* xf = reinterpret_cast<float4*>(xs);
-            xf[((size_t)t * 8 + 2 * q4) * C + c] = a;
-            xf[((size_t)t * 8 + 2 * q4 + 1) * C + c] = b;
-        } else {
-            xs[((size_t)t * 4 + q4) * C + c] = raw;
-        }
+        uint4 o;  // pairs (x0,x4) (x1,x5) (x2,x6) (x3,x7) of these 8 values
+        o.x = __byte_perm(raw.x, raw.z, 0x5410);
+        o.y = __byte_perm(raw.x, raw.z, 0x7632);
+        o.z = __byte_perm(raw.y, raw.w, 0x5410);
+        o.w = __byte_perm(raw.y, raw.w, 0x7632);
+        xs[((size_t)t * 4 + wi) * C + c] = o;
     }
     __syncthreads();
     for (int v = threadIdx.x; v < M * C; v += kThreads) {
         const int t = v / C, c = v - t * C;
-        float s = 0.0f;
-        if (XF32) {
-            const float4* xf = reinterpret_cast<const float4*>(xs);
+        float acc = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 a = xf[((size_t)t * 8 + i) * C + c];
-                s += a.x; s += a.y; s += a.z; s += a.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 a = xs[((size_t)t * 4 + i) * C + c];
-                s += __uint_as_float(a.x << 16); s += __uint_as_float(a.x & 0xFFFF0000u);
-                s += __uint_as_float(a.y << 16); s += __uint_as_float(a.y & 0xFFFF0000u);
-                s += __uint_as_float(a.z << 16); s += __uint_as_float(a.z & 0xFFFF0000u);
-                s += __uint_as_float(a.w << 16); s += __uint_as_float(a.w & 0xFFFF0000u);
-            }
+        for (int wi = 0; wi < 4; ++wi) {
+            const uint4 p = xs[((size_t)t * 4 + wi) * C + c];
+            acc += bf16_lo(p.x); acc += bf16_lo(p.y); acc += bf16_lo(p.z); acc += bf16_lo(p.w);
+            acc += bf16_hi(p.x); acc += bf16_hi(p.y); acc += bf16_hi(p.z); acc += bf16_hi(p.w);
         }
-        sx[v] = s;
+        sx[v] = acc;
     }
     __syncthreads();
+    pdl_launch_dependents();
 
-    const int hw = threadIdx.x >> 4;   // half-warp in CTA
-    const int j = threadIdx.x & 15;    // lane in half-warp
-    const int rows_per_cta = kHalfWarps * RH;
-    const int nblocks = (N + rows_per_cta - 1) / rows_per_cta;
-    const size_t row_bytes = (size_t)(K >> 1);
-
-    for (int blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
-        int rows[RH];
-#pragma unroll
-        for (int i = 0; i < RH; ++i) {
-            const int n = blk * rows_per_cta + hw * RH + i;
-            rows[i] = n < N ? n : N - 1;  // tail rows re-read row N-1; results dropped
-        }
+    for (; blk < nblocks; blk += gridDim.x) {
         float yacc[M][RH];
 #pragma unroll
         for (int t = 0; t < M; ++t)
 #pragma unroll
             for (int i = 0; i < RH; ++i) yacc[t][i] = 0.0f;
-
-        for (int c0 = j; c0 < C; c0 += 16 * U) {
-            uint4 wq[U][RH];
-            float dv[U][RH], mv[U][RH];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 16 * u;
-                const bool live = c < C;
-                const int g = (live ? c : 0) >> 3;
-#pragma unroll
-                for (int i = 0; i < RH; ++i) {
-                    wq[u][i] = live ? ld_nc_v4(codes + rows[i] * row_bytes + (size_t)c * 16)
-                                    : make_uint4(0, 0, 0, 0);
-                    dv[u][i] = live ? ld_f16_as_f32(d + (size_t)rows[i] * G + g) : 0.0f;
-                    mv[u][i] = live ? ld_f16_as_f32(m + (size_t)rows[i] * G + g) : 0.0f;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 16 * u;
-                if (c >= C) break;
-                float a[M][RH];
-#pragma unroll
-                for (int t = 0; t < M; ++t)
-#pragma unroll
-                    for (int i = 0; i < RH; ++i) a[t][i] = 0.0f;
-#pragma unroll
-                for (int wi = 0; wi < 4; ++wi) {
-                    float xv[M][8];
-#pragma unroll
-                    for (int t = 0; t < M; ++t) {
-                        if (XF32) {
-                            const float4* xf = reinterpret_cast<const float4*>(xs);
-                            const float4 p = xf[((size_t)t * 8 + 2 * wi) * C + c];
-                            const float4 q = xf[((size_t)t * 8 + 2 * wi + 1) * C + c];
-                            xv[t][0] = p.x; xv[t][1] = p.y; xv[t][2] = p.z; xv[t][3] = p.w;
-                            xv[t][4] = q.x; xv[t][5] = q.y; xv[t][6] = q.z; xv[t][7] = q.w;
-                        } else {
-                            const uint4 p = xs[((size_t)t * 4 + wi) * C + c];
-                            xv[t][0] = __uint_as_float(p.x << 16);
-                            xv[t][1] = __uint_as_float(p.x & 0xFFFF0000u);
-                            xv[t][2] = __uint_as_float(p.y << 16);
-                            xv[t][3] = __uint_as_float(p.y & 0xFFFF0000u);
-                            xv[t][4] = __uint_as_float(p.z << 16);
-                            xv[t][5] = __uint_as_float(p.z & 0xFFFF0000u);
-                            xv[t][6] = __uint_as_float(p.w << 16);
-                            xv[t][7] = __uint_as_float(p.w & 0xFFFF0000u);
-                        }
-                    }
-#pragma unroll
-                    for (int i = 0; i < RH; ++i) {
-                        const uint32_t w = wi == 0 ? wq[u][i].x
-                                         : wi == 1 ? wq[u][i].y
-                                         : wi == 2 ? wq[u][i].z
-                                                   : wq[u][i].w;
-                        float f[8];
-                        f[0] = nib_f<0>(w); f[1] = nib_f<1>(w); f[2] = nib_f<2>(w);
-                        f[3] = nib_f<3>(w); f[4] = nib_f<4>(w); f[5] = nib_f<5>(w);
-                        f[6] = nib_f<6>(w); f[7] = nib_f<7>(w);
-#pragma unroll
-                        for (int t = 0; t < M; ++t)
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) a[t][i] = fmaf(xv[t][e], f[e], a[t][i]);
-                    }
-                }
-#pragma unroll
-                for (int t = 0; t < M; ++t) {
-                    const float s = sx[t * C + c];
-#pragma unroll
-                    for (int i = 0; i < RH; ++i) {
-                        const float dd = dv[u][i] * 16.0f;
-                        yacc[t][i] = fmaf(dd, a[t][i] - s, fmaf(mv[u][i], s, yacc[t][i]));
-                    }
-                }
+        if (active) {
+            for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
+                if (c0 != cs + j) load_batch(bt, codes, d, m, rows, row_bytes, G, c0, ce);
+                consume_batch<M, RH, U>(bt, xs, sx, C, c0, ce, yacc);
             }
         }
         // reduce the 16 lanes of the half-warp (xor < 16 stays inside it)
@@ -221,33 +267,81 @@ __global__ void __launch_bounds__(kThreads) w4_gemv_kernel(
                 v += __shfl_xor_sync(0xffffffffu, v, 1);
                 yacc[t][i] = v;
             }
-        // lane (t*RH + i) of the half-warp stores element (t, i)
+        // next row block's first batch goes out before the store/reduction
+        const int nblk = blk + gridDim.x;
+        int nrows[RH];
 #pragma unroll
-        for (int t = 0; t < M; ++t)
+        for (int i = 0; i < RH; ++i) {
+            const int n = nblk * rows_per_cta + (active ? rg : 0) * RH + i;
+            nrows[i] = n < N ? n : N - 1;
+        }
+        if (nblk < nblocks && active)
+            load_batch(bt, codes, d, m, nrows, row_bytes, G, cs + j, ce);
+
+        if (KS == 1) {
 #pragma unroll
-            for (int i = 0; i < RH; ++i) {
-                if (j == ((t * RH + i) & 15)) {
-                    const int n = blk * rows_per_cta + hw * RH + i;
-                    if (n < N) {
-                        if (out_f32)
-                            reinterpret_cast<float*>(y)[(size_t)t * N + n] = yacc[t][i];
-                        else
-                            reinterpret_cast<__nv_bfloat16*>(y)[(size_t)t * N + n] =
-                                __float2bfloat16_rn(yacc[t][i]);
+            for (int t = 0; t < M; ++t)
+#pragma unroll
+                for (int i = 0; i < RH; ++i) {
+                    if (active && j == ((t * RH + i) & 15)) {
+                        const int n = blk * rows_per_cta + rg * RH + i;
+                        if (n < N) {
+                            if (out_f32)
+                                reinterpret_cast<float*>(y)[(size_t)t * N + n] = yacc[t][i];
+                            else
+                                reinterpret_cast<__nv_bfloat16*>(y)[(size_t)t * N + n] =
+                                    __float2bfloat16_rn(yacc[t][i]);
+                        }
                     }
                 }
+        } else {
+            if (active && j == 0) {
+#pragma unroll
+                for (int i = 0; i < RH; ++i)
+#pragma unroll
+                    for (int t = 0; t < M; ++t)
+                        red[((size_t)s * rows_per_cta + rg * RH + i) * M + t] = yacc[t][i];
             }
+            __syncthreads();
+            for (int e = threadIdx.x; e < rows_per_cta * M; e += kThreads) {
+                const int r = e / M, t = e - r * M;
+                float v = 0.0f;
+                for (int q = 0; q < KS; ++q) v += red[((size_t)q * rows_per_cta + r) * M + t];
+                const int n = blk * rows_per_cta + r;
+                if (n < N) {
+                    if (out_f32)
+                        reinterpret_cast<float*>(y)[(size_t)t * N + n] = v;
+                    else
+                        reinterpret_cast<__nv_bfloat16*>(y)[(size_t)t * N + n] =
+                            __float2bfloat16_rn(v);
+                }
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int i = 0; i < RH; ++i) rows[i] = nrows[i];
     }
 }
 
-template <int M, int RH, int U, bool XF32>
-int launch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
+size_t smem_bytes(int M, int C, int KS, int RH) {
+    const int rows_per_cta = (kHalfWarps / KS) * RH;
+    return (size_t)M * 4 * C * 16 + (size_t)M * C * 4 +
+           (KS > 1 ? (size_t)KS * rows_per_cta * M * 4 : 0);
+}
+
+template <int M, int RH>
+int launch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K, int KS,
            const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
-    auto kern = w4_gemv_kernel<M, RH, U, XF32>;
+    constexpr int U = 8 / RH;
+    auto kern = w4_gemv_kernel<M, RH, U>;
     const int C = K / 32;
-    const size_t smem = (size_t)M * (XF32 ? 8 : 4) * C * 16 + (size_t)M * C * 4;
+    const size_t smem = smem_bytes(M, C, KS, RH);
     // Per-instantiation cache: one device, a few shared-memory sizes.
-    struct Entry { int dev; size_t smem; int per_sm; };
+    struct Entry {
+        int dev;
+        size_t smem;
+        int per_sm;
+    };
     static thread_local Entry cache[8];
     static thread_local int ncache = 0;
     static thread_local int attr_dev = -1;
@@ -271,34 +365,51 @@ int launch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, in
         cache[ncache & 7] = Entry{dev, smem, per_sm};
         if (ncache < 8) ++ncache;
     }
-    const int rows_per_cta = kHalfWarps * RH;
+    const int rows_per_cta = (kHalfWarps / KS) * RH;
     const int nblocks = (N + rows_per_cta - 1) / rows_per_cta;
     int grid = per_sm * w4::sm_count();
     if (grid > nblocks) grid = nblocks;
-    kern<<<grid, kThreads, smem, st>>>(codes, reinterpret_cast<const __half*>(d),
-                                      reinterpret_cast<const __half*>(m), N, K, x, y, out_f32);
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, codes, reinterpret_cast<const __half*>(d),
+                           reinterpret_cast<const __half*>(m), N, K, KS, x, y, out_f32);
+    if (e != cudaSuccess) return w4::cuda_fail(e);
     return w4::launch_status();
+}
+
+// Rows per half-warp and K-split: enough independent half-warp streams to
+// cover the SMs (~64 per SM), each K-slice at least one chunk per lane.
+void pick_split(int N, int C, int sms, int* rh, int* ks) {
+    const long long target = (long long)sms * 64;
+    if ((long long)N / 4 >= target) { *rh = 4; *ks = 1; return; }
+    if ((long long)N / 2 >= target) { *rh = 2; *ks = 1; return; }
+    *rh = 1;
+    int k = 1;
+    while (k < 16 && (long long)N * k < target && C / (2 * k) >= 16) k *= 2;
+    *ks = k;
 }
 
 template <int M>
 int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
-    const int C = K / 32;
-    const bool f32 = (size_t)M * 8 * C * 16 + (size_t)M * C * 4 <= (size_t)kSmemBudget;
-    // rows per half-warp: enough row-blocks to cover the SMs, else fewer rows
-    // per half-warp (more independent streams).
-    const int sms = w4::sm_count();
-    const bool big = N >= 16 * 4 * sms * 2;
-    if (M <= 2) {
-        if (big) return f32 ? launch<M, 4, 2, true>(codes, d, m, N, K, x, y, out_f32, st)
-                            : launch<M, 4, 2, false>(codes, d, m, N, K, x, y, out_f32, st);
-        return f32 ? launch<M, 1, 8, true>(codes, d, m, N, K, x, y, out_f32, st)
-                   : launch<M, 1, 8, false>(codes, d, m, N, K, x, y, out_f32, st);
+    int rh, ks;
+    pick_split(N, K / 32, w4::sm_count(), &rh, &ks);
+    if (M >= 4 && rh > 2) rh = 2;  // register budget: M * RH accumulators twice
+    if (smem_bytes(M, K / 32, ks, rh) > (size_t)kSmemBudget) ks = 1;
+    if constexpr (M < 4) {
+        if (rh == 4) return launch<M, 4>(codes, d, m, N, K, ks, x, y, out_f32, st);
     }
-    if (big) return f32 ? launch<M, 2, 2, true>(codes, d, m, N, K, x, y, out_f32, st)
-                        : launch<M, 2, 2, false>(codes, d, m, N, K, x, y, out_f32, st);
-    return f32 ? launch<M, 1, 4, true>(codes, d, m, N, K, x, y, out_f32, st)
-               : launch<M, 1, 4, false>(codes, d, m, N, K, x, y, out_f32, st);
+    if (rh >= 2) return launch<M, 2>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    return launch<M, 1>(codes, d, m, N, K, ks, x, y, out_f32, st);
 }
 
 }  // namespace
@@ -308,14 +419,13 @@ extern "C" int w4_gemv(const uint8_t* codes, const uint16_t* d_f16, const uint16
                        int out_dtype, void* stream) {
     if (M < 1 || M > 8 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
     if (N > (int64_t)1 << 30 || K > (int64_t)1 << 20) return W4_ERR_SHAPE;
-    if (N * (K / 2) > ((int64_t)1 << 40)) return W4_ERR_SHAPE;
     if (out_dtype != W4_OUT_BF16 && out_dtype != W4_OUT_F32) return W4_ERR_SHAPE;
     if (!codes || !d_f16 || !m_f16 || !x_bf16 || !y) return W4_ERR_NULL;
     if (!w4::aligned16(codes) || !w4::aligned16(d_f16) || !w4::aligned16(m_f16) ||
         !w4::aligned16(x_bf16) || !w4::aligned16(y))
         return W4_ERR_ALIGN;
-    // x must fit shared memory at least as bf16 (M * K * 2 bytes + sums)
-    if ((int64_t)M * K * 2 + (int64_t)M * (K / 32) * 4 > kSmemBudget) return W4_ERR_SHAPE;
+    // x (M*K bf16) and its chunk sums must fit the shared-memory stage
+    if (smem_bytes(M, (int)(K / 32), 1, 1) > (size_t)kSmemBudget) return W4_ERR_SHAPE;
     int rc = w4::check_device();
     if (rc != W4_OK) return rc;
     const int out_f32 = out_dtype == W4_OUT_F32;

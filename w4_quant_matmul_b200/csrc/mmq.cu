@@ -9,25 +9,41 @@
 //   y[t][n]    = sum_g ( d[n][g] * sum_{b in g} dx[t][b] * P[t][n][b]
 //                        + m[n][g] * sum_{b in g} dx[t][b] * S[t][b] )
 //
-// One CTA computes a 128 (tokens) x 128 (weight rows) tile of y, looping over
-// K in stages of 128 (four 32-element activation blocks):
+// One CTA computes a 128 (tokens) x 128 (weight rows) tile of y over a range
+// of K (all of it, or one of S slices when the grid would not fill the SMs),
+// in pipeline stages of 128 (four 32-element activation blocks):
 //   warp 0      TMA producer: the qa tile (128 x 128 B, 128B-swizzled) and the
 //               packed code tile (128 rows x 64 B) into a 4-stage ring.
 //   warp 1      allocates 512 TMEM columns; one lane issues, per 32-block, one
 //               tcgen05.mma.kind::i8 (M=128, N=128, K=32; A = qa as s8, B = the
-//               codes as u8) into its own 128-column TMEM buffer, overwriting
-//               it, so every block's exact int32 products stay separate.
+//               codes as u8) into its own 128-column TMEM buffer, so every
+//               block's exact int32 products stay separate.
 //   warps 2-3   unpack each code tile, nibble -> byte, into the 128B-swizzled
 //               K-major layout the MMA's shared-memory descriptor expects
 //               (tcgen05 has no 4-bit integer kind).
 //   warps 4-11  epilogue: each thread owns one token row (its TMEM lane) and 64
-//               weight rows; per block it loads the 64 int32 products, releases
-//               the buffer, and accumulates dx[t][b] * P into a per-group sum;
-//               at each group end it applies d[n][g] and the exact min term
-//               m[n][g] * sum_b dx[t][b] S[t][b].
+//               weight rows.
+//
+// Epilogue arithmetic.  Converting 16384 int32 products per block to float at
+// the quarter-rate conversion throughput would cost four times the MMA, so
+// no conversion is done: every TMEM buffer holds the integer bias 65536
+// before its MMA, which accumulates onto it (|P| <= 32*15*127 = 60960), so
+// the word read back is V = 65536 + P in [4576, 126496] -- as fp32 bits, the
+// exact denormal V * 2^-149.  With dx scaled by a power of two 2^e chosen per
+// (token, group) so that products stay normal, one full-rate FMA per element
+// accumulates acc = sum_b (dx_b 2^e) V_b 2^-149, and at the group end
+//   sum_b dx_b P_b = acc * 2^(149-e) - 65536 * sum_b dx_b
+// (one FMA, a single rounding), then y += d * that + m * sum_b dx_b S_b.
+// After loading a buffer the epilogue writes the bias back (tcgen05.st) before
+// releasing it to the MMA.  Requires |dx| < 2^100 (activations far beyond
+// any fp16/bf16 model range would overflow the scaled products).
+//
 // The MMA runs up to four blocks ahead of the epilogue (four TMEM buffers).
 // Registers are rebalanced with setmaxnreg: 72 per thread for warps 0-3, 216
 // for the epilogue (128*72 + 256*216 = 384*168, the launch allotment).
+// K slices (split-K) write fp32 partial tiles to the caller's workspace; the
+// CTA that finishes a tile last sums the partials in slice order (bitwise
+// deterministic) and stores y.
 // Every mbarrier wait is bounded; a wait that runs out raises the CTA's abort
 // flag and the device error word, all roles drain what they issued, TMEM is
 // freed and the CTA returns.
@@ -76,7 +92,12 @@ struct Params {
     int M, N, K;
     int out_f32;
     int* err;
+    int splits;            // K slices per output tile (1 = no split)
+    int* counters;         // [tiles] arrival counters (split > 1), zeroed before launch
+    float* partials;       // [tiles][splits][BM][BN] fp32 partial tiles
 };
+
+constexpr uint32_t kBias = 65536u;  // TMEM accumulators start at this integer
 
 // ---------------------------------------------------------------------------
 // tcgen05 wrappers
@@ -131,6 +152,20 @@ __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 consecutive columns of this warp's 32 lanes <- v.
+__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // kernel
 // ---------------------------------------------------------------------------
@@ -162,7 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * BN;
     const int m0 = blockIdx.y * BM;
-    const int ksteps = p.K / BK;
+    // K slice of this CTA, in whole groups (two stages per 256-group)
+    const int ngroups = p.K / 256;
+    const int g_begin = (int)(((long long)ngroups * blockIdx.z) / p.splits);
+    const int g_end = (int)(((long long)ngroups * (blockIdx.z + 1)) / p.splits);
+    const int ks_begin = g_begin * 2;
+    const int ksteps = (g_end - g_begin) * 2;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -218,8 +258,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
                     if (!w4::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err)) break;
                     w4::mbar_arrive_expect_tx(&full[s], A_BYTES + BP_BYTES);
-                    w4::tma_load_2d(sa + s * A_BYTES, &tm_a, &full[s], ks * BK, m0);
-                    w4::tma_load_2d(sbp + s * BP_BYTES, &tm_b, &full[s], ks * (BK / 2), n0);
+                    const int kg = ks_begin + ks;
+                    w4::tma_load_2d(sa + s * A_BYTES, &tm_a, &full[s], kg * BK, m0);
+                    w4::tma_load_2d(sbp + s * BP_BYTES, &tm_b, &full[s], kg * (BK / 2), n0);
                     issued = ks + 1;
                 }
                 // drain: every issued load must land before the CTA exits
@@ -245,14 +286,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t b_addr = w4::smem_u32(sb + s * B_BYTES);
                     bool ok = true;
                     for (int q = 0; q < NBUF; ++q) {
-                        if (!w4::mbar_wait(&tempty[q], ((uint32_t)ks & 1u) ^ 1u, abort_flag,
-                                           p.err)) {
+                        // phase ks of tempty[q]: the epilogue has (re)filled the
+                        // buffer with the bias (phase 0: the initial fill)
+                        if (!w4::mbar_wait(&tempty[q], (uint32_t)ks & 1u, abort_flag, p.err)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         mma_i8(tmem_base + (uint32_t)(q * BN), smem_desc_sw128(a_addr + q * KB),
-                               smem_desc_sw128(b_addr + q * KB), idesc, 0u);
+                               smem_desc_sw128(b_addr + q * KB), idesc, 1u);
                         mma_commit(&tfull[q]);
                     }
                     mma_commit(&empty[s]);
@@ -299,84 +341,160 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool t_live = t < p.M;
         const int B = p.K / KB;
         const uint32_t tm_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(h * 64);
+        // initial bias fill of the four buffers = phase 0 of tempty[q]
+#pragma unroll 1
+        for (int q = 0; q < NBUF; ++q) {
+            tmem_fill32(tm_row + (uint32_t)(q * BN), kBias);
+            tmem_fill32(tm_row + (uint32_t)(q * BN + 32), kBias);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            for (int q = 0; q < NBUF; ++q) w4::mbar_arrive(&tempty[q]);
+
         float acc[64], yv[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
             acc[c] = 0.0f;
             yv[c] = 0.0f;
         }
-        float dxg[8];
-        float tmin = 0.0f;
+        float pe = 0.0f;           // 2^e of the current group
+        const float* dx_row = p.dx + (size_t)(t_live ? t : 0) * B;
+        float kpow = 0.0f;         // 2^(149 - e)
+        float neg_bias = 0.0f;     // -65536 * sum_b dx_b
+        float tmin = 0.0f;         // sum_b dx_b * S_b
         bool ok = true;
         for (int ks = 0; ks < ksteps && ok; ++ks) {
 #pragma unroll 1
             for (int q = 0; q < NBUF; ++q) {
-                const int kb = ks * NBUF + q;
-                const int g = kb >> 3;
+                const int kb = ks * NBUF + q;         // block index within the slice
+                const int g = g_begin + (kb >> 3);    // global group index
                 if ((kb & 7) == 0) {
-                    // activation scales and block sums of this group (32-byte aligned)
+                    float dxg[8];
+                    int sg[8];
                     if (t_live) {
-                        const float4* dp = reinterpret_cast<const float4*>(p.dx + (size_t)t * B + g * 8);
+                        const float4* dp =
+                            reinterpret_cast<const float4*>(p.dx + (size_t)t * B + g * 8);
                         const int4* sp = reinterpret_cast<const int4*>(p.S + (size_t)t * B + g * 8);
                         const float4 a0 = __ldg(dp), a1 = __ldg(dp + 1);
                         const int4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
                         dxg[0] = a0.x; dxg[1] = a0.y; dxg[2] = a0.z; dxg[3] = a0.w;
                         dxg[4] = a1.x; dxg[5] = a1.y; dxg[6] = a1.z; dxg[7] = a1.w;
-                        tmin = dxg[0] * (float)s0.x;
-                        tmin = fmaf(dxg[1], (float)s0.y, tmin);
-                        tmin = fmaf(dxg[2], (float)s0.z, tmin);
-                        tmin = fmaf(dxg[3], (float)s0.w, tmin);
-                        tmin = fmaf(dxg[4], (float)s1.x, tmin);
-                        tmin = fmaf(dxg[5], (float)s1.y, tmin);
-                        tmin = fmaf(dxg[6], (float)s1.z, tmin);
-                        tmin = fmaf(dxg[7], (float)s1.w, tmin);
+                        sg[0] = s0.x; sg[1] = s0.y; sg[2] = s0.z; sg[3] = s0.w;
+                        sg[4] = s1.x; sg[5] = s1.y; sg[6] = s1.z; sg[7] = s1.w;
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) dxg[i] = 0.0f;
-                        tmin = 0.0f;
+                        for (int i = 0; i < 8; ++i) {
+                            dxg[i] = 0.0f;
+                            sg[i] = 0;
+                        }
                     }
+                    float dmax = 0.0f, usum = 0.0f;
+                    tmin = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        dmax = fmaxf(dmax, dxg[i]);
+                        usum += dxg[i];
+                        tmin = fmaf(dxg[i], (float)sg[i], tmin);
+                    }
+                    // e: dmax * 2^e in [2^40, 2^41), clamped to [22, 127]
+                    const int ex = (int)((__float_as_uint(dmax) >> 23) & 0xFFu);
+                    int e = 167 - ex;
+                    e = e < 22 ? 22 : (e > 127 ? 127 : e);
+                    pe = __uint_as_float((uint32_t)(e + 127) << 23);
+                    kpow = __uint_as_float((uint32_t)(149 - e + 127) << 23);
+                    neg_bias = -65536.0f * usum;
                 }
                 if (!w4::mbar_wait(&tfull[q], (uint32_t)ks & 1u, abort_flag, p.err)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tm_row + (uint32_t)(q * BN), r0);
-                tmem_ld32(tm_row + (uint32_t)(q * BN + 32), r1);
-                tmem_wait_ld();
+                // dx_b * 2^e (exact power-of-two scaling); 0 for rows past M
+                const float sc = t_live ? __ldg(dx_row + g_begin * 8 + kb) * pe : 0.0f;
+                // two 32-column halves: load, refill with the bias, accumulate
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t r[32];
+                    const uint32_t ta = tm_row + (uint32_t)(q * BN + 32 * hh);
+                    tmem_ld32(ta, r);
+                    tmem_wait_ld();
+                    tmem_fill32(ta, kBias);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        acc[32 * hh + c] = fmaf(sc, __uint_as_float(r[c]), acc[32 * hh + c]);
+                }
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) w4::mbar_arrive(&tempty[q]);
-                float dxb = dxg[0];
-#pragma unroll
-                for (int i = 1; i < 8; ++i)
-                    if ((kb & 7) == i) dxb = dxg[i];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    acc[c] = fmaf(dxb, (float)(int)r0[c], acc[c]);
-                    acc[32 + c] = fmaf(dxb, (float)(int)r1[c], acc[32 + c]);
-                }
                 if ((kb & 7) == 7) {
-                    const float4* dg = reinterpret_cast<const float4*>(d_s + g * BN + h * 64);
-                    const float4* mg = reinterpret_cast<const float4*>(m_s + g * BN + h * 64);
+                    const int gl = g;  // d_s/m_s hold every group of the row block
+                    const float4* dg = reinterpret_cast<const float4*>(d_s + gl * BN + h * 64);
+                    const float4* mg = reinterpret_cast<const float4*>(m_s + gl * BN + h * 64);
 #pragma unroll
                     for (int c4 = 0; c4 < 16; ++c4) {
                         const float4 dv = dg[c4], mv = mg[c4];
-                        yv[4 * c4 + 0] = fmaf(dv.x, acc[4 * c4 + 0], fmaf(mv.x, tmin, yv[4 * c4 + 0]));
-                        yv[4 * c4 + 1] = fmaf(dv.y, acc[4 * c4 + 1], fmaf(mv.y, tmin, yv[4 * c4 + 1]));
-                        yv[4 * c4 + 2] = fmaf(dv.z, acc[4 * c4 + 2], fmaf(mv.z, tmin, yv[4 * c4 + 2]));
-                        yv[4 * c4 + 3] = fmaf(dv.w, acc[4 * c4 + 3], fmaf(mv.w, tmin, yv[4 * c4 + 3]));
-                        acc[4 * c4 + 0] = 0.0f;
-                        acc[4 * c4 + 1] = 0.0f;
-                        acc[4 * c4 + 2] = 0.0f;
-                        acc[4 * c4 + 3] = 0.0f;
+                        const float dvv[4] = {dv.x, dv.y, dv.z, dv.w};
+                        const float mvv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const int c = 4 * c4 + e4;
+                            const float a = fmaf(acc[c], kpow, neg_bias);
+                            yv[c] = fmaf(dvv[e4], a, fmaf(mvv[e4], tmin, yv[c]));
+                            acc[c] = 0.0f;
+                        }
                     }
                 }
             }
         }
-        if (ok && t_live) {
-            const int nb = n0 + h * 64;
+        // ---- store: directly, or through the split-K workspace ----
+        const int nb = n0 + h * 64;
+        bool store = ok && t_live;
+        if (p.splits > 1) {
+            // Every epilogue thread reaches both barriers, aborted or not.
+            const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+            if (ok) {
+                float* mine =
+                    p.partials + (((size_t)tile * p.splits + blockIdx.z) * BM + row) * BN + h * 64;
+#pragma unroll
+                for (int c4 = 0; c4 < 16; ++c4)
+                    *reinterpret_cast<float4*>(mine + 4 * c4) =
+                        make_float4(yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
+            }
+            __threadfence();
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            volatile int* last_flag = abort_flag + 1;
+            if (threadIdx.x == 128) {
+                int last = 0;
+                if (!*abort_flag) last = atomicAdd(p.counters + tile, 1) == p.splits - 1;
+                *last_flag = last;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            const bool last = *last_flag != 0;
+            store = store && last;
+            if (last) {
+                __threadfence();
+                const float* base =
+                    p.partials + ((size_t)tile * p.splits * BM + row) * BN + h * 64;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) yv[c] = 0.0f;
+                for (int q = 0; q < p.splits; ++q) {
+                    const float4* src = reinterpret_cast<const float4*>(base + (size_t)q * BM * BN);
+#pragma unroll
+                    for (int c4 = 0; c4 < 16; ++c4) {
+                        const float4 v = __ldcg(src + c4);
+                        yv[4 * c4] += v.x;
+                        yv[4 * c4 + 1] += v.y;
+                        yv[4 * c4 + 2] += v.z;
+                        yv[4 * c4 + 3] += v.w;
+                    }
+                }
+                if (threadIdx.x == 128) p.counters[tile] = 0;  // ready for the next call
+            }
+        }
+        if (store) {
             if (p.out_f32) {
                 float* yr = reinterpret_cast<float*>(p.y) + (size_t)t * p.N;
                 if (nb + 64 <= p.N && (p.N & 3) == 0) {
@@ -461,22 +579,51 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K slices per output tile.  Cost model in units of one 256-group of MMA work
+// per CTA: waves(tiles * S over the SMs) * (groups per slice + fixed cost of a
+// CTA's fill, drain and epilogue), each slice keeping >= 4 groups.
+int pick_splits(int64_t M, int64_t N, int64_t K, int sms) {
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int G = (int)(K / 256);
+    int best = 1;
+    double best_cost = 1e30;
+    for (int sp = 1; sp <= 16 && sp <= G; ++sp) {
+        if (sp > 1 && G / sp < 4) break;
+        const int64_t waves = (tiles * sp + sms - 1) / sms;
+        const double cost = (double)waves * ((double)G / sp + 1.5) + (sp > 1 ? 0.25 * sp : 0.0);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = sp;
+        }
+    }
+    return best;
+}
+
+constexpr size_t kCounterBytesAlign = 256;
+
+size_t counters_bytes(int64_t tiles) {
+    return ((size_t)tiles * 4 + kCounterBytesAlign - 1) / kCounterBytesAlign * kCounterBytesAlign;
+}
+
+size_t workspace_for(int64_t M, int64_t N, int64_t K, int splits) {
+    if (splits <= 1) return 0;
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    return counters_bytes(tiles) + (size_t)tiles * splits * BM * BN * sizeof(float);
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K) {
-    (void)M;
-    (void)N;
-    (void)K;
-    return 0;
+    if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return 0;
+    (void)w4::check_device();  // fills the SM count when a device is present
+    return workspace_for(M, N, K, pick_splits(M, N, K, w4::sm_count()));
 }
 
 int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
              int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
              void* y, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
-    (void)workspace;
-    (void)ws_bytes;
     if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
     if (K / 256 > kMaxGroups || M > (1 << 24) || N > (1 << 24)) return W4_ERR_SHAPE;
     if (out_dtype != W4_OUT_BF16 && out_dtype != W4_OUT_F32) return W4_ERR_SHAPE;
@@ -488,6 +635,13 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     if (rc != W4_OK) return rc;
     int* err = w4::device_error_word();
     if (!err) return W4_ERR_CUDA;
+    const int splits = pick_splits(M, N, K, w4::sm_count());
+    const size_t need = workspace_for(M, N, K, splits);
+    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    if (need > 0) {
+        if (!workspace || ws_bytes < need) return W4_ERR_WORKSPACE;
+        if (!w4::aligned16(workspace)) return W4_ERR_ALIGN;
+    }
 
     CUtensorMap ma, mb;
     if (!make_map_u8(&ma, qa, (uint64_t)K, (uint64_t)M, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -519,7 +673,17 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     prm.K = (int)K;
     prm.out_f32 = out_dtype == W4_OUT_F32;
     prm.err = err;
-    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM));
+    prm.splits = splits;
+    prm.counters = nullptr;
+    prm.partials = nullptr;
+    if (splits > 1) {
+        prm.counters = static_cast<int*>(workspace);
+        prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                                counters_bytes(tiles));
+        e = cudaMemsetAsync(workspace, 0, (size_t)tiles * 4, (cudaStream_t)stream);
+        if (e != cudaSuccess) return w4::cuda_fail(e);
+    }
+    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM), (unsigned)splits);
     w4a8_mmq_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, prm);
     return w4::launch_status();
 }
