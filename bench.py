@@ -235,6 +235,7 @@ class Workload:
                 .to(self.dev).view(torch.bfloat16) for i, (N, K) in enumerate(SHAPES)]
             self.y[M] = [torch.empty((M, N), dtype=torch.bfloat16, device=self.dev)
                          for (N, K) in SHAPES]
+            torch.cuda.synchronize()
         return self.x[M], self.y[M]
 
 
@@ -330,6 +331,11 @@ def time_e2e(torch, w4, wl, steps, warmup, stream):
 def time_mmq(torch, w4, dev, stream, reps=5):
     """W4A8 prefill product at M = 256..2048 on both prefill shapes, plus the
     activation quantiser.  Returns a list of result dicts."""
+    with torch.cuda.stream(stream):  # every torch op below is ordered on `stream`
+        return _time_mmq(torch, w4, dev, stream, reps)
+
+
+def _time_mmq(torch, w4, dev, stream, reps):
     out = []
     g = torch.Generator(device=dev)
     g.manual_seed(11)
@@ -343,11 +349,13 @@ def time_mmq(torch, w4, dev, stream, reps=5):
                 synth.CONFIG_MMQ, si)).view(np.int16)).to(dev).view(torch.bfloat16)
             qa, dx, S = w4.q8_quantize_act(x, stream=stream)
             y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            torch.cuda.synchronize()
             for _ in range(3):
                 w4.w4a8_mmq(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y, stream=stream)
             tq, tm = [], []
             for _ in range(reps):
-                flush.zero_()
+                with torch.cuda.stream(stream):
+                    flush.zero_()  # L2 flush, ordered before the timed launches
                 e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
                 e0.record(stream)
                 w4.q8_quantize_act(x, qa, dx, S, stream=stream)

@@ -77,6 +77,20 @@ def test_degenerate_weights(torch, w4, orc):
     _both(torch, w4, orc, codes, d, m, x, what="degenerate")
 
 
+def test_activation_outliers_and_dynamic_range(torch, w4, orc):
+    # the kernel holds each 32-element activation chunk as 16-bit fixed point
+    # relative to the chunk's largest magnitude: sparse x20 outliers and
+    # elements spanning 12 decades must stay inside the gate
+    N, K = 300, 2560
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=40)
+    x1 = synth.outlier_activations(4, K, seed=41)
+    rng = np.random.default_rng(42)
+    wide = (rng.standard_normal((4, K)) * 10.0 ** rng.uniform(-6, 3, size=(4, K)))
+    x2 = synth.f32_to_bf16_bits(wide.astype(np.float32))
+    for x in (x1, x2):
+        _both(torch, w4, orc, codes, d, m, x, what="outliers/range")
+
+
 @pytest.mark.parametrize("shape_index", range(len(synth.GEMV_SHAPES)))
 def test_full_size_sampled_rows(torch, w4, orc, shape_index):
     N, K = synth.GEMV_SHAPES[shape_index]

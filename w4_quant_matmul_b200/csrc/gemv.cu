@@ -5,35 +5,40 @@
 //   y[t][n] = sum_g ( d[n][g] * sum_{k in g} q[n][k] x[t][k]
 //                     + m[n][g] * sum_{k in g} x[t][k] )
 //
-// HBM-bound at M = 1 (0.515625 weight bytes per multiply-add), so the design
-// goal is a weight stream that keeps enough bytes in flight and an inner loop
-// cheap enough not to become the limit:
+// HBM-bound at M = 1 (0.515625 weight bytes per multiply-add); on B200 the
+// CUDA-core instruction issue rate, not the FMA rate, is what a dequant-fused
+// GEMV runs into first, so the inner loop is built on integer dot products:
 //
+//  * Activations, per 32-element chunk (once per CTA, in shared memory): the
+//    chunk's largest exponent E fixes sigma = 2^(14 - E), and every element
+//    becomes the 16-bit integer X = rint(x * sigma), split X = 256 Xh + Xl
+//    (Xh signed, Xl unsigned bytes).  Every element within a factor 2^7 of
+//    the chunk's largest magnitude is represented exactly (bf16 carries 8
+//    significant bits); smaller ones are rounded with an absolute error of at
+//    most 2^-15 of the chunk's largest magnitude.  The chunk sum Sx of the
+//    original values (fp32, fixed order) is kept for the min term.
+//  * Weights: a code word (8 nibbles) splits into the bytes of its low and
+//    high nibbles with three logic ops; dp4a multiplies four codes by four
+//    activation bytes and accumulates in int32, so 8 codes cost 3 logic ops +
+//    4 dp4a per token, and sum_k q X is exact: 256 * sum(q Xh) + sum(q Xl)
+//    (|.| <= 32 * 15 * 32640 < 2^24, exact in fp32 too).  Per chunk
+//        sum q x ~= (sum q X) / sigma,    y += d * that + m * Sx.
 //  * Work split.  A half-warp (16 lanes) owns RH rows and one of KS K-slices;
 //    lane j streams the 16-byte code chunks (32 codes) c = j, j+16, ... of its
 //    slice with non-allocating 128-bit loads, U chunks ahead per row.  With
 //    KS > 1 the slices of a row are summed in fixed order through shared
 //    memory (small-N shapes need the extra streams); with KS = 1 a 4-step
-//    xor-shuffle finishes the row.  CTAs loop over row blocks.
-//  * Dequantisation.  Two codes at a time become a bf16x2 pair (128 + q) by
-//    OR-ing their nibbles, shifted to bits 0-3 of each half, into the bf16
-//    exponent of 128: one logic op for k and k+4 of a word, a shift and a logic
-//    op for the other three pairs.  The mixed-precision fma.rn.f32.bf16 then
-//    accumulates x * (128 + q) in fp32 at full FMA rate, exactly (8-bit x 8-bit
-//    products), so per 32-code chunk
-//        A = sum x (128 + q)   and   sum q x = A - 128 * Sx,
-//    and the chunk adds d (A - 128 Sx) + m Sx (Sx = sum of its 32 x).
-//  * Activations.  x is staged once per CTA into shared memory as bf16 pairs
-//    permuted to match the code pairs, chunk-minor (sub-word w of chunk c at
-//    [w][c]) so the 16 lanes of a half-warp hit 16 different banks; the chunk
-//    sums Sx are staged beside them (fp32, fixed order).
+//    xor-shuffle finishes the row.  CTAs loop over row blocks.  The staged
+//    activation words are chunk-minor ([word][chunk]) so the 16 lanes of a
+//    half-warp read 16 different banks.
 //  * Programmatic dependent launch.  Before griddepcontrol.wait the CTA only
 //    asks L2 to prefetch its first batch of weights (bulk L2 prefetch; L2 is
 //    the point of coherence, so a prefetch can never observe stale data even
 //    if the preceding kernel writes the weights).  In a chain of launches the
 //    first HBM round trip of this GEMV overlaps the tail of the previous
 //    kernel; every load that feeds arithmetic happens after the wait.
-// Accumulation is fp32 in a fixed order: results are bitwise deterministic.
+// Integer sums are exact and the float reductions run in a fixed order:
+// results are bitwise deterministic.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -59,25 +64,6 @@ __device__ __forceinline__ uint16_t ld_nc_u16(const void* p) {
     return r;
 }
 
-// acc += lo(xp) * lo(fp) + hi(xp) * hi(fp), each product exact, fp32 accumulate.
-__device__ __forceinline__ float fma_bf16x2(uint32_t xp, uint32_t fp, float acc) {
-    asm("{\n\t.reg .b16 xl, xh, fl, fh;\n\t"
-        "mov.b32 {xl, xh}, %1;\n\t"
-        "mov.b32 {fl, fh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, xl, fl, %0;\n\t"
-        "fma.rn.f32.bf16 %0, xh, fh, %0;\n\t}\n"
-        : "+f"(acc)
-        : "r"(xp), "r"(fp));
-    return acc;
-}
-
-// bf16x2 (128 + q_lo, 128 + q_hi) from the nibbles at bits [s, s+4) and
-// [s+16, s+20) of a code word.
-template <int S>
-__device__ __forceinline__ uint32_t code_pair(uint32_t w) {
-    return ((w >> S) & 0x000F000Fu) | 0x43004300u;
-}
-
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
@@ -94,7 +80,7 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 template <int RH, int U>
 struct Batch {
     uint4 wq[U][RH];
-    uint16_t dv[U][RH], mv[U][RH];
+    uint32_t dm[U][RH];
 };
 
 template <int RH, int U>
@@ -111,75 +97,140 @@ __device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __res
         for (int i = 0; i < RH; ++i) {
             if (live) {
                 b.wq[u][i] = ld_nc_v4(codes + rows[i] * row_bytes + (size_t)c * 16);
-                b.dv[u][i] = ld_nc_u16(d + (size_t)rows[i] * G + g);
-                b.mv[u][i] = ld_nc_u16(m + (size_t)rows[i] * G + g);
+                b.dm[u][i] = (uint32_t)ld_nc_u16(d + (size_t)rows[i] * G + g) |
+                             ((uint32_t)ld_nc_u16(m + (size_t)rows[i] * G + g) << 16);
             } else {
                 b.wq[u][i] = make_uint4(0, 0, 0, 0);
-                b.dv[u][i] = 0;
-                b.mv[u][i] = 0;
+                b.dm[u][i] = 0;
             }
         }
     }
 }
 
 template <int M, int RH, int U>
-__device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4* __restrict__ xs,
-                                              const float* __restrict__ sx, int C, int c0,
+__device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4* __restrict__ xq,
+                                              const float* __restrict__ sx,
+                                              const float* __restrict__ inv, int C, int c0,
                                               int c_end, float (&yacc)[M][RH]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int c = c0 + 16 * u;
         if (c >= c_end) break;
-        float a[M][RH];
+        int ah[M][RH], al[M][RH];
 #pragma unroll
         for (int t = 0; t < M; ++t)
 #pragma unroll
-            for (int i = 0; i < RH; ++i) a[t][i] = 0.0f;
+            for (int i = 0; i < RH; ++i) {
+                ah[t][i] = 0;
+                al[t][i] = 0;
+            }
 #pragma unroll
         for (int wi = 0; wi < 4; ++wi) {
-            uint4 xv[M];
+            uint4 xv[M];  // {Xh even k, Xh odd k, Xl even k, Xl odd k} of this word
 #pragma unroll
-            for (int t = 0; t < M; ++t) xv[t] = xs[((size_t)t * 4 + wi) * C + c];
+            for (int t = 0; t < M; ++t) xv[t] = xq[((size_t)t * 4 + wi) * C + c];
 #pragma unroll
             for (int i = 0; i < RH; ++i) {
                 const uint32_t w = wi == 0 ? b.wq[u][i].x
                                  : wi == 1 ? b.wq[u][i].y
                                  : wi == 2 ? b.wq[u][i].z
                                            : b.wq[u][i].w;
-                const uint32_t f0 = code_pair<0>(w), f1 = code_pair<4>(w);
-                const uint32_t f2 = code_pair<8>(w), f3 = code_pair<12>(w);
+                const uint32_t lo = w & 0x0F0F0F0Fu;         // codes of k = 0, 2, 4, 6
+                const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // codes of k = 1, 3, 5, 7
 #pragma unroll
                 for (int t = 0; t < M; ++t) {
-                    a[t][i] = fma_bf16x2(xv[t].x, f0, a[t][i]);
-                    a[t][i] = fma_bf16x2(xv[t].y, f1, a[t][i]);
-                    a[t][i] = fma_bf16x2(xv[t].z, f2, a[t][i]);
-                    a[t][i] = fma_bf16x2(xv[t].w, f3, a[t][i]);
+                    ah[t][i] = __dp4a((int)lo, (int)xv[t].x, ah[t][i]);
+                    ah[t][i] = __dp4a((int)hi, (int)xv[t].y, ah[t][i]);
+                    al[t][i] = (int)__dp4a(lo, xv[t].z, (unsigned)al[t][i]);
+                    al[t][i] = (int)__dp4a(hi, xv[t].w, (unsigned)al[t][i]);
                 }
             }
         }
 #pragma unroll
         for (int t = 0; t < M; ++t) {
-            const float s = sx[t * C + c];
+            const float s = sx[t * C + c], iv = inv[t * C + c];
 #pragma unroll
             for (int i = 0; i < RH; ++i) {
-                const float dd = __half2float(__ushort_as_half(b.dv[u][i]));
-                const float mm = __half2float(__ushort_as_half(b.mv[u][i]));
-                yacc[t][i] = fmaf(dd, fmaf(-128.0f, s, a[t][i]), fmaf(mm, s, yacc[t][i]));
+                const float dd = __half2float(__ushort_as_half((unsigned short)(b.dm[u][i] & 0xFFFFu)));
+                const float mm = __half2float(__ushort_as_half((unsigned short)(b.dm[u][i] >> 16)));
+                const float qx = (float)(ah[t][i] * 256 + al[t][i]) * iv;
+                yacc[t][i] = fmaf(dd, qx, fmaf(mm, s, yacc[t][i]));
             }
         }
     }
 }
 
+// One quarter (8 values) of a 32-element activation chunk -> its activation
+// word; lanes 4q..4q+3 of a warp hold the four quarters of one chunk.  Writes
+// the word and (lane quarter 0) the chunk sum and 1/sigma.  Every lane of the
+// warp must call it (the chunk reductions are xor-shuffles); `live` = false
+// lanes contribute nothing and store nothing.
+__device__ __forceinline__ void stage_quarter(uint4 raw, bool live, uint4* __restrict__ word_dst,
+                                              float* __restrict__ sum_dst,
+                                              float* __restrict__ inv_dst, int quarter) {
+    float f[8] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y),
+                  bf16_lo(raw.z), bf16_hi(raw.z), bf16_lo(raw.w), bf16_hi(raw.w)};
+    float s = 0.0f;
+    uint32_t emax = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        s += f[e];
+        emax = max(emax, (__float_as_uint(f[e]) >> 23) & 0xFFu);
+    }
+    // fixed-order chunk sum: (q0 + q1) + (q2 + q3)
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, 1));
+    emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, 2));
+    // sigma = 2^(14 - E) with E = emax - 127, as an exponent field in [1, 253]
+    int se = 268 - (int)emax;
+    se = se < 1 ? 1 : (se > 253 ? 253 : se);
+    const float sigma = __uint_as_float((uint32_t)se << 23);
+    int X[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        // rint(f * sigma) exactly: f * sigma is exact and |.| < 2^15, so adding
+        // 1.5 * 2^23 rounds to the nearest integer, which sits in the mantissa
+        const float t = fmaf(f[e], sigma, 12582912.0f);
+        X[e] = emax == 0 ? 0 : (int)(__float_as_uint(t) - 0x4B400000u);
+    }
+    // bytes: even k -> (X0, X2, X4, X6), odd k -> (X1, X3, X5, X7)
+    const uint32_t e01 = __byte_perm((uint32_t)X[0], (uint32_t)X[2], 0x0040);
+    const uint32_t e23 = __byte_perm((uint32_t)X[4], (uint32_t)X[6], 0x0040);
+    const uint32_t o01 = __byte_perm((uint32_t)X[1], (uint32_t)X[3], 0x0040);
+    const uint32_t o23 = __byte_perm((uint32_t)X[5], (uint32_t)X[7], 0x0040);
+    const uint32_t eh01 = __byte_perm((uint32_t)X[0], (uint32_t)X[2], 0x0051);
+    const uint32_t eh23 = __byte_perm((uint32_t)X[4], (uint32_t)X[6], 0x0051);
+    const uint32_t oh01 = __byte_perm((uint32_t)X[1], (uint32_t)X[3], 0x0051);
+    const uint32_t oh23 = __byte_perm((uint32_t)X[5], (uint32_t)X[7], 0x0051);
+    if (live) {
+        *word_dst = make_uint4(__byte_perm(eh01, eh23, 0x5410), __byte_perm(oh01, oh23, 0x5410),
+                               __byte_perm(e01, e23, 0x5410), __byte_perm(o01, o23, 0x5410));
+        if (quarter == 0) {
+            *sum_dst = s;
+            *inv_dst = emax == 0 ? 0.0f : __uint_as_float((uint32_t)(254 - se) << 23);
+        }
+    }
+}
+
+// Resident CTAs per SM the register allocation is sized for: small M needs
+// many warps in flight to cover HBM latency; large M needs the registers.
+template <int M>
+struct MinCtas {
+    static constexpr int value = M == 1 ? 3 : (M <= 4 ? 2 : 1);
+};
+
 template <int M, int RH, int U>
-__global__ void __launch_bounds__(kThreads) w4_gemv_kernel(
+__global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
     int N, int K, int KS, const uint16_t* __restrict__ x, void* __restrict__ y, int out_f32) {
     extern __shared__ __align__(16) unsigned char smem[];
     const int C = K >> 5;  // 32-code chunks per row
     const int G = K >> 8;  // groups per row
-    uint4* xs = reinterpret_cast<uint4*>(smem);                                // [M][4][C]
+    uint4* xq = reinterpret_cast<uint4*>(smem);                                // [M][4][C]
     float* sx = reinterpret_cast<float*>(smem + (size_t)M * 4 * C * 16);         // [M][C]
-    float* red = sx + (size_t)M * C;  // [KS][rows_per_cta][M] partial sums (KS > 1)
+    float* inv = sx + (size_t)M * C;                                             // [M][C]
+    float* red = inv + (size_t)M * C;  // [KS][rows_per_cta][M] partial sums (KS > 1)
 
     const int hw = threadIdx.x >> 4;  // half-warp in CTA
     const int j = threadIdx.x & 15;   // lane in half-warp
@@ -211,37 +262,24 @@ __global__ void __launch_bounds__(kThreads) w4_gemv_kernel(
 
     // ---- everything below may depend on the previous kernel in the stream ----
     pdl_wait();
-    Batch<RH, U> bt;
-    if (blk < nblocks && active) load_batch(bt, codes, d, m, rows, row_bytes, G, cs + j, ce);
 
-    // ---- x and its chunk sums, once per CTA ----
-    const int nvec = M * C * 4;  // uint4 (8 bf16) units of x
-    for (int v = threadIdx.x; v < nvec; v += kThreads) {
-        const int t = v / (C * 4);
-        const int r = v - t * C * 4;
-        const int c = r >> 2, wi = r & 3;
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(x) + v);
-        uint4 o;  // pairs (x0,x4) (x1,x5) (x2,x6) (x3,x7) of these 8 values
-        o.x = __byte_perm(raw.x, raw.z, 0x5410);
-        o.y = __byte_perm(raw.x, raw.z, 0x7632);
-        o.z = __byte_perm(raw.y, raw.w, 0x5410);
-        o.w = __byte_perm(raw.y, raw.w, 0x7632);
-        xs[((size_t)t * 4 + wi) * C + c] = o;
-    }
-    __syncthreads();
-    for (int v = threadIdx.x; v < M * C; v += kThreads) {
-        const int t = v / C, c = v - t * C;
-        float acc = 0.0f;
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-            const uint4 p = xs[((size_t)t * 4 + wi) * C + c];
-            acc += bf16_lo(p.x); acc += bf16_lo(p.y); acc += bf16_lo(p.z); acc += bf16_lo(p.w);
-            acc += bf16_hi(p.x); acc += bf16_hi(p.y); acc += bf16_hi(p.z); acc += bf16_hi(p.w);
-        }
-        sx[v] = acc;
+    // ---- activation words, chunk sums and scales, once per CTA ----
+    const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
+    for (int base = 0; base < nq; base += kThreads) {
+        const int v = base + threadIdx.x;
+        const bool live = v < nq;
+        const int vv = live ? v : 0;
+        const int t = vv / (C * 4);
+        const int r = vv - t * C * 4;
+        const int c = r >> 2, q4 = r & 3;
+        const uint4 raw = live ? __ldg(reinterpret_cast<const uint4*>(x) + vv) : make_uint4(0, 0, 0, 0);
+        stage_quarter(raw, live, &xq[((size_t)t * 4 + q4) * C + c], &sx[t * C + c],
+                      &inv[t * C + c], q4);
     }
     __syncthreads();
     pdl_launch_dependents();
+    Batch<RH, U> bt;
+    if (blk < nblocks && active) load_batch(bt, codes, d, m, rows, row_bytes, G, cs + j, ce);
 
     for (; blk < nblocks; blk += gridDim.x) {
         float yacc[M][RH];
@@ -252,7 +290,7 @@ __global__ void __launch_bounds__(kThreads) w4_gemv_kernel(
         if (active) {
             for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
                 if (c0 != cs + j) load_batch(bt, codes, d, m, rows, row_bytes, G, c0, ce);
-                consume_batch<M, RH, U>(bt, xs, sx, C, c0, ce, yacc);
+                consume_batch<M, RH, U>(bt, xq, sx, inv, C, c0, ce, yacc);
             }
         }
         // reduce the 16 lanes of the half-warp (xor < 16 stays inside it)
@@ -325,7 +363,7 @@ __global__ void __launch_bounds__(kThreads) w4_gemv_kernel(
 
 size_t smem_bytes(int M, int C, int KS, int RH) {
     const int rows_per_cta = (kHalfWarps / KS) * RH;
-    return (size_t)M * 4 * C * 16 + (size_t)M * C * 4 +
+    return (size_t)M * 4 * C * 16 + (size_t)M * C * 8 +
            (KS > 1 ? (size_t)KS * rows_per_cta * M * 4 : 0);
 }
 
