@@ -145,6 +145,35 @@ int w4a8_mmq(const uint8_t *codes, const uint16_t *d_f16,
              const float *dx, const int32_t *bsum, int64_t M, void *y,
              int out_dtype, void *workspace, size_t ws_bytes, void *stream);
 
+/* Size of the library-owned device scratch behind w4a8_mmq_static. */
+#define W4A8_MMQ_STATIC_SCRATCH_BYTES (40u * 1024u * 1024u)
+
+/* The W4A8 product of w4a8_mmq for callers that cannot allocate device memory
+ * (the pages have no counterpart: this entry point exists for the library's
+ * users, not for the method).  Some callers cannot call cudaMalloc or hand out
+ * a workspace: code that runs while a CUDA graph is being captured, plugins
+ * whose host framework owns every allocation, and deployments with a fixed
+ * memory plan decided before the first request.  This entry point takes the
+ * same inputs and output as w4a8_mmq but no workspace: the split-K scratch is a
+ * static device array owned by the library, W4A8_MMQ_STATIC_SCRATCH_BYTES
+ * (40 MiB) on every GPU that loads libw4, kept until the process exits.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - A shape whose scratch need (w4a8_mmq_workspace_size) exceeds the static
+ *     size is rejected with W4_ERR_WORKSPACE before anything is enqueued (use
+ *     w4a8_mmq with a caller workspace for it).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it: make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last call's
+ *     contents (the arrival counters it needs at zero are cleared on the call's
+ *     stream): calls that can overlap on the GPU -- on different streams, or
+ *     from several host threads -- race on it and must be serialised.
+ * Arguments, layouts and results are those of w4a8_mmq. */
+int w4a8_mmq_static(const uint8_t *codes, const uint16_t *d_f16,
+                    const uint16_t *m_f16, int64_t N, int64_t K,
+                    const int8_t *qa, const float *dx, const int32_t *bsum,
+                    int64_t M, void *y, int out_dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,6 +13,7 @@ Entry points (same names as the C ABI):
     w4_gemv(codes, d, m, x, out_dtype)      -> y
     q8_quantize_act(x)                      -> qa, dx, bsum
     w4a8_mmq(codes, d, m, qa, dx, bsum, out_dtype) -> y
+    w4a8_mmq_static(codes, d, m, qa, dx, bsum, out_dtype) -> y   (no workspace)
     w4a8_mmq_workspace_size(M, N, K)
     w4_check_device_error()
 """
@@ -22,7 +23,8 @@ from ._lib import (LibraryMissing, W4_OK, W4_OUT_BF16, W4_OUT_F32, load, status_
 
 __all__ = [
     "W4Error", "LibraryMissing", "w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv",
-    "q8_quantize_act", "w4a8_mmq", "w4a8_mmq_workspace_size", "w4_check_device_error",
+    "q8_quantize_act", "w4a8_mmq", "w4a8_mmq_static", "w4a8_mmq_workspace_size",
+    "w4_check_device_error",
     "w4_abi_version", "lib",
 ]
 
@@ -207,4 +209,28 @@ def w4a8_mmq(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, workspace=None, 
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(load().w4a8_mmq(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(qa), _ptr(dx), _ptr(bsum),
                            M, _ptr(y), oc, ws_ptr, ws_bytes, _stream(stream)), "w4a8_mmq")
+    return y
+
+
+def w4a8_mmq_static(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, stream=None):
+    """The W4A8 product without a workspace, for callers that cannot allocate
+    device memory: the split-K scratch is the library's static device array
+    (shared by every call on the device; overlapping calls must be serialised).
+    Raises W4Error (W4_ERR_WORKSPACE) for shapes whose scratch need exceeds it."""
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    _need(codes, torch.uint8, "codes")
+    _need(d, torch.float16, "d")
+    _need(m, torch.float16, "m")
+    _need(qa, torch.int8, "qa")
+    _need(dx, torch.float32, "dx")
+    _need(bsum, torch.int32, "bsum")
+    N = codes.shape[0]
+    M, K = qa.shape
+    oc = _out_code(out_dtype)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32 if oc == W4_OUT_F32 else torch.bfloat16,
+                        device=qa.device)
+    _check(load().w4a8_mmq_static(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(qa), _ptr(dx),
+                                  _ptr(bsum), M, _ptr(y), oc, _stream(stream)), "w4a8_mmq_static")
     return y

@@ -40,7 +40,10 @@ SIGNATURES = {
     "w4a8_mmq_workspace_size": ([_I64, _I64, _I64], ctypes.c_size_t),
     "w4a8_mmq": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P, ctypes.c_size_t, _P],
                  _INT),
+    "w4a8_mmq_static": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P], _INT),
 }
+
+W4A8_MMQ_STATIC_SCRATCH_BYTES = 40 * 1024 * 1024
 
 
 class LibraryMissing(RuntimeError):

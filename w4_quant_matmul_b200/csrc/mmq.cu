@@ -689,3 +689,56 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// w4a8_mmq_static: the same product for callers that cannot allocate device
+// memory.  The split-K scratch lives in a library-owned static device array
+// instead of a caller workspace.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// Every GPU that loads this library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_mmq_static_scratch[W4A8_MMQ_STATIC_SCRATCH_BYTES];
+
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kStaticMaxDevices];
+
+// Device address of the static scratch on the current device.  The host-side
+// name of a __device__ array is only a stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+int static_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return w4::cuda_fail(e);
+    if (dev < 0 || dev >= kStaticMaxDevices) return W4_ERR_UNSUPPORTED_DEVICE;
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_mmq_static_scratch);
+        if (e != cudaSuccess) return w4::cuda_fail(e);
+        g_static_addr[dev] = p;
+    }
+    *out = g_static_addr[dev];
+    return W4_OK;
+}
+
+}  // namespace
+
+extern "C" int w4a8_mmq_static(const uint8_t* codes, const uint16_t* d_f16,
+                               const uint16_t* m_f16, int64_t N, int64_t K, const int8_t* qa,
+                               const float* dx, const int32_t* bsum, int64_t M, void* y,
+                               int out_dtype, void* stream) {
+    if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
+    int rc = w4::check_device();
+    if (rc != W4_OK) return rc;
+    const size_t need = w4a8_mmq_workspace_size(M, N, K);
+    if (need > (size_t)W4A8_MMQ_STATIC_SCRATCH_BYTES) return W4_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if (need > 0) {
+        rc = static_scratch(&ws);
+        if (rc != W4_OK) return rc;
+    }
+    return w4a8_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype, ws, need, stream);
+}
