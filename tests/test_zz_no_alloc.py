@@ -65,8 +65,13 @@ def test_static_scratch_matches_workspace_entry_point(torch, lib, orc):
 
 def test_static_scratch_rejects_oversized_shapes(torch, lib):
     from w4_quant_matmul_b200 import _lib
-    M, N, K = 1024, 2560, 9728
-    assert lib.w4a8_mmq_workspace_size(M, N, K) > _lib.W4A8_MMQ_STATIC_SCRATCH_BYTES
+    # the first split-K shape whose scratch need exceeds the static array
+    # (the need depends on the tile shape, so it is asked of the library)
+    over = [(M, N, K) for M, N, K in [(1024, 2560, 9728), (1024, 4096, 14336),
+                                      (1536, 2560, 14336), (2048, 4096, 14336)]
+            if lib.w4a8_mmq_workspace_size(M, N, K) > _lib.W4A8_MMQ_STATIC_SCRATCH_BYTES]
+    assert over, "no candidate shape exceeds the static scratch"
+    M, N, K = over[0]
     buf = torch.zeros(16, dtype=torch.uint8, device="cuda")
     p = _ptr(buf)  # never read: the size check comes first
     rc = lib.w4a8_mmq_static(p, p, p, N, K, p, p, p, M, p, _lib.W4_OUT_F32, None)

@@ -9,9 +9,10 @@
 //   y[t][n]    = sum_g ( d[n][g] * sum_{b in g} dx[t][b] * P[t][n][b]
 //                        + m[n][g] * sum_{b in g} dx[t][b] * S[t][b] )
 //
-// One CTA computes a 128 (tokens) x 128 (weight rows) tile of y over a range
-// of K (all of it, or one of S slices when the grid would not fill the SMs),
-// in pipeline stages of 128 (four 32-element activation blocks):
+// Persistent CTAs (one per SM) loop over work units = (128-token x 128-row
+// output tile, K slice); the pipeline, barriers and TMEM allocation live for
+// the whole launch.  K advances in stages of 128 (four 32-element activation
+// blocks):
 //   warp 0      TMA producer: the qa tile (128 x 128 B, 128B-swizzled) and the
 //               packed code tile (128 rows x 64 B) into a 4-stage ring.
 //   warp 1      allocates 512 TMEM columns; one lane issues, per 32-block, one
@@ -22,21 +23,26 @@
 //               K-major layout the MMA's shared-memory descriptor expects
 //               (tcgen05 has no 4-bit integer kind).
 //   warps 4-11  epilogue: each thread owns one token row (its TMEM lane) and 64
-//               weight rows.
+//               weight rows.  Per block it loads its 64 words with one wait,
+//               refills the bias and releases the buffer before any arithmetic,
+//               so the MMA only waits on TMEM round trips, not on the FMAs.
 //
 // Epilogue arithmetic.  Converting 16384 int32 products per block to float at
 // the quarter-rate conversion throughput would cost four times the MMA, so
-// no conversion is done: every TMEM buffer holds the integer bias 65536
-// before its MMA, which accumulates onto it (|P| <= 32*15*127 = 60960), so
-// the word read back is V = 65536 + P in [4576, 126496] -- as fp32 bits, the
-// exact denormal V * 2^-149.  With dx scaled by a power of two 2^e chosen per
-// (token, group) so that products stay normal, one full-rate FMA per element
-// accumulates acc = sum_b (dx_b 2^e) V_b 2^-149, and at the group end
+// no conversion is done: before each block's MMA the tensor core writes the
+// integer bias 65536 into the block's TMEM buffer (a second kind::i8 MMA over
+// constant u8 tiles, 32 * 32 * 64 = 65536, in overwrite mode), and the block's
+// MMA accumulates onto it (|P| <= 32*15*127 = 60960), so the word read back
+// is V = 65536 + P in [4576, 126496] -- as fp32 bits, the exact denormal
+// V * 2^-149.  With dx scaled by a power of two 2^e chosen per (token, group)
+// so that products stay normal, one full-rate FMA per element accumulates
+// acc = sum_b (dx_b 2^e) V_b 2^-149, and at the group end
 //   sum_b dx_b P_b = acc * 2^(149-e) - 65536 * sum_b dx_b
 // (one FMA, a single rounding), then y += d * that + m * sum_b dx_b S_b.
-// After loading a buffer the epilogue writes the bias back (tcgen05.st) before
-// releasing it to the MMA.  Requires |dx| < 2^100 (activations far beyond
-// any fp16/bf16 model range would overflow the scaled products).
+// The TMEM-to-register path (about 340 B per SM per clock on B200, measured)
+// is what bounds this kernel: every block's 128 x 128 int32 products must be
+// read once.  Requires |dx| < 2^100 (activations far beyond any fp16/bf16
+// model range would overflow the scaled products).
 //
 // The MMA runs up to four blocks ahead of the epilogue (four TMEM buffers).
 // Registers are rebalanced with setmaxnreg: 72 per thread for warps 0-3, 216
@@ -62,13 +68,17 @@ constexpr int BN = 128;        // weight rows per tile (MMA N)
 constexpr int BK = 128;        // K elements per pipeline stage
 constexpr int KB = 32;         // activation block = MMA K for kind::i8
 constexpr int STAGES = 4;
-constexpr int NBUF = BK / KB;  // TMEM buffers, one per block of a stage
-constexpr int kThreads = 384;
+constexpr int NBLK = BK / KB;  // 32-blocks per pipeline stage
+constexpr int NTB = 4;         // TMEM block buffers (BN columns each)
+constexpr int BIAS_BYTES = 128 * KB;  // one constant operand tile of the bias MMA
+constexpr int kThreads = 384;              // 4 producer-side warps + 8 epilogue warps
+constexpr int kEpiWarps = 8;
+constexpr int kEpiCols = BN / (kEpiWarps / 4); // 64 weight rows per epilogue thread
 constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BN * BK;
 constexpr int BP_BYTES = BN * BK / 2;
-constexpr int TMEM_COLS = NBUF * BN;  // 512
-constexpr int kMaxGroups = 64;        // K <= 16384
+constexpr int TMEM_COLS = NTB * BN;   // 512
+constexpr int kMaxGroups = 56;        // K <= 14336 (shared memory for d, m)
 
 static_assert(TMEM_COLS == 512, "TMEM allocation must be a power of two <= 512");
 
@@ -76,8 +86,9 @@ struct Smem {
     static constexpr int a = 0;
     static constexpr int b = a + STAGES * A_BYTES;
     static constexpr int bp = b + STAGES * B_BYTES;
-    static constexpr int bars = bp + STAGES * BP_BYTES;  // uint64 barriers
-    static constexpr int nbars = 3 * STAGES + 2 * NBUF + 1;
+    static constexpr int bias = bp + STAGES * BP_BYTES;  // bias MMA operands (A, B)
+    static constexpr int bars = bias + 2 * BIAS_BYTES;   // uint64 barriers
+    static constexpr int nbars = 3 * STAGES + 2 * NTB + 1;
     static constexpr int misc = bars + nbars * 8;        // tmem base, abort flag
     static constexpr int dm = (misc + 16 + 15) & ~15;    // fp32 d[G][BN], m[G][BN]
     static size_t total(int G) { return (size_t)dm + (size_t)2 * G * BN * 4 + 1024; }
@@ -93,11 +104,12 @@ struct Params {
     int out_f32;
     int* err;
     int splits;            // K slices per output tile (1 = no split)
+    int tiles_n;           // output tiles along N
+    int units;             // tiles * splits work units (CTAs loop over them)
     int* counters;         // [tiles] arrival counters (split > 1), zeroed before launch
     float* partials;       // [tiles][splits][BM][BN] fp32 partial tiles
 };
 
-constexpr uint32_t kBias = 65536u;  // TMEM accumulators start at this integer
 
 // ---------------------------------------------------------------------------
 // tcgen05 wrappers
@@ -114,6 +126,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
     // K-major, 128-byte swizzle: 8-row core groups 1024 bytes apart.
     return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
            ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// K-major, no swizzle, for the 128 x 32-byte constant tiles of the bias MMA:
+// 8-row x 16-byte core matrices, K-neighbours 128 B apart, 8-row groups 256 B
+// apart (every byte of these tiles is equal, so only the extent matters).
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t addr) {
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 16) |
+           ((uint64_t)(256 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
 __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -152,20 +172,6 @@ __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 32 consecutive columns of this warp's 32 lanes <- v.
-__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
-        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};" ::"r"(taddr),
-        "r"(v)
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() {
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------
 // kernel
 // ---------------------------------------------------------------------------
@@ -185,24 +191,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* unpacked = bars + STAGES;      // B unpacked into the MMA layout
     uint64_t* empty = bars + 2 * STAGES;     // MMAs of the stage done
     uint64_t* tfull = bars + 3 * STAGES;     // TMEM buffer written
-    uint64_t* tempty = tfull + NBUF;         // TMEM buffer drained
-    uint64_t* drain = tempty + NBUF;         // final MMA completion
+    uint64_t* tempty = tfull + NTB;          // TMEM buffer drained and refilled
+    uint64_t* drain = tempty + NTB;          // final MMA completion
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Smem::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
+    volatile int* last_flag = abort_flag + 1;
     float* d_s = reinterpret_cast<float*>(smem + Smem::dm);
     const int G = p.K / 256;
     float* m_s = d_s + G * BN;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;
-    const int m0 = blockIdx.y * BM;
-    // K slice of this CTA, in whole groups (two stages per 256-group)
-    const int ngroups = p.K / 256;
-    const int g_begin = (int)(((long long)ngroups * blockIdx.z) / p.splits);
-    const int g_end = (int)(((long long)ngroups * (blockIdx.z + 1)) / p.splits);
-    const int ks_begin = g_begin * 2;
-    const int ksteps = (g_end - g_begin) * 2;
+    const int ngroups = G;
+
+    // Work unit u -> (tile_m, tile_n, K slice).  Units handed to consecutive
+    // CTAs share tile_m, i.e. the same activation rows.
+    auto unit_of = [&](int u, int& tm, int& tn, int& gb, int& ge) {
+        const int split = u % p.splits;
+        const int tile = u / p.splits;
+        tn = tile % p.tiles_n;
+        tm = tile / p.tiles_n;
+        gb = (int)(((long long)ngroups * split) / p.splits);
+        ge = (int)(((long long)ngroups * (split + 1)) / p.splits);
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -210,13 +221,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             w4::mbar_init(&unpacked[i], 2);
             w4::mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < NBUF; ++i) {
+        for (int i = 0; i < NTB; ++i) {
             w4::mbar_init(&tfull[i], 1);
-            w4::mbar_init(&tempty[i], 8);
+            w4::mbar_init(&tempty[i], kEpiWarps);
         }
         w4::mbar_init(drain, 1);
         *abort_flag = 0;
         w4::fence_mbar_init();
+    }
+    // constant operands of the bias MMA: A = 32, B = 64 (u8), so that over K = 32
+    // every accumulator starts at 32 * 32 * 64 = 65536
+    {
+        uint32_t* ba = reinterpret_cast<uint32_t*>(smem + Smem::bias);
+        for (int i = threadIdx.x; i < 2 * BIAS_BYTES / 4; i += kThreads)
+            ba[i] = i < BIAS_BYTES / 4 ? 0x20202020u : 0x40404040u;
+        w4::fence_proxy_async_smem();
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -224,21 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                      "r"(TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    // epilogue threads stage this tile's d and m (fp32, [g][n]); rows past N -> 0
-    if (warp >= 4) {
-        const int e = threadIdx.x - 128;
-        for (int i = e; i < BN * G; i += 256) {
-            const int r = i / G, g = i - r * G;
-            const int n = n0 + r;
-            float dv = 0.0f, mv = 0.0f;
-            if (n < p.N) {
-                dv = __half2float(p.d[(size_t)n * G + g]);
-                mv = __half2float(p.m[(size_t)n * G + g]);
-            }
-            d_s[g * BN + r] = dv;
-            m_s[g * BN + r] = mv;
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -252,21 +256,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (w4::elect_one()) {
                 w4::prefetch_tmap(&tm_a);
                 w4::prefetch_tmap(&tm_b);
-                int issued = 0;
-                for (int ks = 0; ks < ksteps; ++ks) {
-                    const int s = ks % STAGES;
-                    const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-                    if (!w4::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err)) break;
-                    w4::mbar_arrive_expect_tx(&full[s], A_BYTES + BP_BYTES);
-                    const int kg = ks_begin + ks;
-                    w4::tma_load_2d(sa + s * A_BYTES, &tm_a, &full[s], kg * BK, m0);
-                    w4::tma_load_2d(sbp + s * BP_BYTES, &tm_b, &full[s], kg * (BK / 2), n0);
-                    issued = ks + 1;
+                int it = 0;  // global stage counter
+                bool ok = true;
+                for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+                    int tmi, tni, gb, ge;
+                    unit_of(u, tmi, tni, gb, ge);
+                    for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
+                        const int s = it % STAGES;
+                        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                        if (!w4::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        w4::mbar_arrive_expect_tx(&full[s], A_BYTES + BP_BYTES);
+                        w4::tma_load_2d(sa + s * A_BYTES, &tm_a, &full[s], kg * BK, tmi * BM);
+                        w4::tma_load_2d(sbp + s * BP_BYTES, &tm_b, &full[s], kg * (BK / 2),
+                                        tni * BN);
+                    }
                 }
                 // drain: every issued load must land before the CTA exits
-                for (int ks = issued - STAGES < 0 ? 0 : issued - STAGES; ks < issued; ++ks)
-                    w4::mbar_wait(&full[ks % STAGES], (uint32_t)(ks / STAGES) & 1u, nullptr,
-                                  p.err);
+                for (int k = it - STAGES < 0 ? 0 : it - STAGES; k < it; ++k)
+                    w4::mbar_wait(&full[k % STAGES], (uint32_t)(k / STAGES) & 1u, nullptr, p.err);
             }
         } else if (warp == 1) {
             // ---------------- MMA issuer ----------------
@@ -276,29 +286,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                                            | (0u << 10)          // B: u8
                                            | ((uint32_t)(BN >> 3) << 17)
                                            | ((uint32_t)(BM >> 4) << 24);
-                for (int ks = 0; ks < ksteps; ++ks) {
-                    const int s = ks % STAGES;
-                    const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-                    if (!w4::mbar_wait(&full[s], ph, abort_flag, p.err)) break;
-                    if (!w4::mbar_wait(&unpacked[s], ph, abort_flag, p.err)) break;
-                    tc_fence_after();
-                    const uint32_t a_addr = w4::smem_u32(sa + s * A_BYTES);
-                    const uint32_t b_addr = w4::smem_u32(sb + s * B_BYTES);
-                    bool ok = true;
-                    for (int q = 0; q < NBUF; ++q) {
-                        // phase ks of tempty[q]: the epilogue has (re)filled the
-                        // buffer with the bias (phase 0: the initial fill)
-                        if (!w4::mbar_wait(&tempty[q], (uint32_t)ks & 1u, abort_flag, p.err)) {
+                constexpr uint32_t idesc_bias = (2u << 4)        // D: s32, A: u8, B: u8
+                                                | ((uint32_t)(BN >> 3) << 17)
+                                                | ((uint32_t)(BM >> 4) << 24);
+                const uint64_t bias_a = smem_desc_plain(w4::smem_u32(smem + Smem::bias));
+                const uint64_t bias_b =
+                    smem_desc_plain(w4::smem_u32(smem + Smem::bias + BIAS_BYTES));
+                int it = 0;
+                bool ok = true;
+                for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+                    int tmi, tni, gb, ge;
+                    unit_of(u, tmi, tni, gb, ge);
+                    for (int kg = gb * 2; kg < ge * 2 && ok; ++kg, ++it) {
+                        const int s = it % STAGES;
+                        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                        if (!w4::mbar_wait(&full[s], ph, abort_flag, p.err) ||
+                            !w4::mbar_wait(&unpacked[s], ph, abort_flag, p.err)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        mma_i8(tmem_base + (uint32_t)(q * BN), smem_desc_sw128(a_addr + q * KB),
-                               smem_desc_sw128(b_addr + q * KB), idesc, 1u);
-                        mma_commit(&tfull[q]);
+                        const uint32_t a_addr = w4::smem_u32(sa + s * A_BYTES);
+                        const uint32_t b_addr = w4::smem_u32(sb + s * B_BYTES);
+                        for (int q = 0; q < NBLK; ++q) {
+                            // block kbg goes to buffer kbg % NTB; wait until the epilogue
+                            // has read that buffer's previous block (first use: free)
+                            const int kbg = it * NBLK + q;
+                            const int b = kbg % NTB;
+                            const uint32_t par = ((uint32_t)(kbg / NTB) & 1u) ^ 1u;
+                            if (!w4::mbar_wait(&tempty[b], par, abort_flag, p.err)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t dt = tmem_base + (uint32_t)(b * BN);
+                            mma_i8(dt, bias_a, bias_b, idesc_bias, 0u);  // D = 65536
+                            mma_i8(dt, smem_desc_sw128(a_addr + q * KB),
+                                   smem_desc_sw128(b_addr + q * KB), idesc, 1u);  // D += P
+                            mma_commit(&tfull[b]);
+                        }
+                        mma_commit(&empty[s]);
                     }
-                    mma_commit(&empty[s]);
-                    if (!ok) break;
                 }
                 mma_commit(drain);
                 w4::mbar_wait(drain, 0u, nullptr, p.err);
@@ -306,227 +334,244 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
             // ---------------- unpackers (warps 2, 3) ----------------
             const int ut = threadIdx.x - 64;  // 0..63
-            for (int ks = 0; ks < ksteps; ++ks) {
-                const int s = ks % STAGES;
-                const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-                if (!w4::mbar_wait(&full[s], ph, abort_flag, p.err)) break;
-                const uint8_t* src = sbp + s * BP_BYTES;
-                uint8_t* dst = sb + s * B_BYTES;
+            int it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+                int tmi, tni, gb, ge;
+                unit_of(u, tmi, tni, gb, ge);
+                for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (!w4::mbar_wait(&full[s], ph, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t* src = sbp + s * BP_BYTES;
+                    uint8_t* dst = sb + s * B_BYTES;
 #pragma unroll 4
-                for (int it = 0; it < (BN * 8) / 64; ++it) {
-                    const int item = it * 64 + ut;
-                    const int r = item >> 3, jc = item & 7;  // row, 16-code chunk
-                    const uint2 pk = *reinterpret_cast<const uint2*>(src + r * (BK / 2) + jc * 8);
-                    const uint32_t lo0 = pk.x & 0x0F0F0F0Fu, hi0 = (pk.x >> 4) & 0x0F0F0F0Fu;
-                    const uint32_t lo1 = pk.y & 0x0F0F0F0Fu, hi1 = (pk.y >> 4) & 0x0F0F0F0Fu;
-                    uint4 o;
-                    o.x = __byte_perm(lo0, hi0, 0x5140);
-                    o.y = __byte_perm(lo0, hi0, 0x7362);
-                    o.z = __byte_perm(lo1, hi1, 0x5140);
-                    o.w = __byte_perm(lo1, hi1, 0x7362);
-                    *reinterpret_cast<uint4*>(dst + r * BK + ((jc ^ (r & 7)) << 4)) = o;
+                    for (int i = 0; i < (BN * 8) / 64; ++i) {
+                        const int item = i * 64 + ut;
+                        const int r = item >> 3, jc = item & 7;  // row, 16-code chunk
+                        const uint2 pk =
+                            *reinterpret_cast<const uint2*>(src + r * (BK / 2) + jc * 8);
+                        const uint32_t lo0 = pk.x & 0x0F0F0F0Fu, hi0 = (pk.x >> 4) & 0x0F0F0F0Fu;
+                        const uint32_t lo1 = pk.y & 0x0F0F0F0Fu, hi1 = (pk.y >> 4) & 0x0F0F0F0Fu;
+                        uint4 o;
+                        o.x = __byte_perm(lo0, hi0, 0x5140);
+                        o.y = __byte_perm(lo0, hi0, 0x7362);
+                        o.z = __byte_perm(lo1, hi1, 0x5140);
+                        o.w = __byte_perm(lo1, hi1, 0x7362);
+                        *reinterpret_cast<uint4*>(dst + r * BK + ((jc ^ (r & 7)) << 4)) = o;
+                    }
+                    w4::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) w4::mbar_arrive(&unpacked[s]);
                 }
-                w4::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) w4::mbar_arrive(&unpacked[s]);
             }
         }
     } else {
         // ---------------- epilogue (warps 4..11) ----------------
         asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+        const int et = threadIdx.x - 128;           // 0..255
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
-        const int h = (warp - 4) >> 2;              // column half: 64 weight rows
+        const int cs = (warp - 4) >> 2;             // column slice: kEpiCols weight rows
         const int row = quarter * 32 + lane;        // token row within the tile
-        const int t = m0 + row;
-        const bool t_live = t < p.M;
         const int B = p.K / KB;
-        const uint32_t tm_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(h * 64);
-        // initial bias fill of the four buffers = phase 0 of tempty[q]
-#pragma unroll 1
-        for (int q = 0; q < NBUF; ++q) {
-            tmem_fill32(tm_row + (uint32_t)(q * BN), kBias);
-            tmem_fill32(tm_row + (uint32_t)(q * BN + 32), kBias);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-            for (int q = 0; q < NBUF; ++q) w4::mbar_arrive(&tempty[q]);
+        const uint32_t tm_row =
+            tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cs * kEpiCols);
 
-        float acc[64], yv[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-            acc[c] = 0.0f;
-            yv[c] = 0.0f;
-        }
-        float pe = 0.0f;           // 2^e of the current group
-        const float* dx_row = p.dx + (size_t)(t_live ? t : 0) * B;
-        float kpow = 0.0f;         // 2^(149 - e)
-        float neg_bias = 0.0f;     // -65536 * sum_b dx_b
-        float tmin = 0.0f;         // sum_b dx_b * S_b
+        int it = 0;
         bool ok = true;
-        for (int ks = 0; ks < ksteps && ok; ++ks) {
+        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+            int tmi, tni, g_begin, g_end;
+            unit_of(u, tmi, tni, g_begin, g_end);
+            const int n0 = tni * BN;
+            const int t = tmi * BM + row;
+            const bool t_live = t < p.M;
+            // this tile's d and m, fp32 [g][n]; rows past N -> 0
+            asm volatile("bar.sync 1, 256;" ::: "memory");  // previous unit done with them
+            for (int i = et; i < BN * (g_end - g_begin); i += 256) {
+                const int r = i / (g_end - g_begin), g = g_begin + (i - r * (g_end - g_begin));
+                const int n = n0 + r;
+                float dv = 0.0f, mv = 0.0f;
+                if (n < p.N) {
+                    dv = __half2float(p.d[(size_t)n * G + g]);
+                    mv = __half2float(p.m[(size_t)n * G + g]);
+                }
+                d_s[g * BN + r] = dv;
+                m_s[g * BN + r] = mv;
+            }
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+
+            float acc[kEpiCols], yv[kEpiCols];
+#pragma unroll
+            for (int c = 0; c < kEpiCols; ++c) {
+                acc[c] = 0.0f;
+                yv[c] = 0.0f;
+            }
+            float pe = 0.0f, kpow = 0.0f, neg_bias = 0.0f, tmin = 0.0f;
+            const float* dx_row = p.dx + (size_t)(t_live ? t : 0) * B;
+            const int ksteps = (g_end - g_begin) * 2;
+            for (int ks = 0; ks < ksteps && ok; ++ks, ++it) {
 #pragma unroll 1
-            for (int q = 0; q < NBUF; ++q) {
-                const int kb = ks * NBUF + q;         // block index within the slice
-                const int g = g_begin + (kb >> 3);    // global group index
-                if ((kb & 7) == 0) {
-                    float dxg[8];
-                    int sg[8];
-                    if (t_live) {
-                        const float4* dp =
-                            reinterpret_cast<const float4*>(p.dx + (size_t)t * B + g * 8);
-                        const int4* sp = reinterpret_cast<const int4*>(p.S + (size_t)t * B + g * 8);
-                        const float4 a0 = __ldg(dp), a1 = __ldg(dp + 1);
-                        const int4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
-                        dxg[0] = a0.x; dxg[1] = a0.y; dxg[2] = a0.z; dxg[3] = a0.w;
-                        dxg[4] = a1.x; dxg[5] = a1.y; dxg[6] = a1.z; dxg[7] = a1.w;
-                        sg[0] = s0.x; sg[1] = s0.y; sg[2] = s0.z; sg[3] = s0.w;
-                        sg[4] = s1.x; sg[5] = s1.y; sg[6] = s1.z; sg[7] = s1.w;
+                for (int q = 0; q < NBLK; ++q) {
+                    const int kb = ks * NBLK + q;         // block index within the slice
+                    const int kbg = it * NBLK + q;        // global block counter
+                    const int b = kbg % NTB;              // its TMEM buffer
+                    const int g = g_begin + (kb >> 3);    // global group index
+                    if ((kb & 7) == 0) {
+                        // group set-up: max, sum and S-weighted sum of the 8 block scales
+                        float dmax = 0.0f, usum = 0.0f;
+                        tmin = 0.0f;
+                        if (t_live) {
+#pragma unroll
+                            for (int h4 = 0; h4 < 2; ++h4) {
+                                const float4 a = __ldg(reinterpret_cast<const float4*>(dx_row + g * 8) + h4);
+                                const int4 sv =
+                                    __ldg(reinterpret_cast<const int4*>(p.S + (size_t)t * B + g * 8) + h4);
+                                dmax = fmaxf(fmaxf(dmax, fmaxf(a.x, a.y)), fmaxf(a.z, a.w));
+                                usum += a.x; usum += a.y; usum += a.z; usum += a.w;
+                                tmin = fmaf(a.x, (float)sv.x, tmin);
+                                tmin = fmaf(a.y, (float)sv.y, tmin);
+                                tmin = fmaf(a.z, (float)sv.z, tmin);
+                                tmin = fmaf(a.w, (float)sv.w, tmin);
+                            }
+                        }
+                        // e: dmax * 2^e in [2^40, 2^41), clamped to [22, 127]
+                        const int ex = (int)((__float_as_uint(dmax) >> 23) & 0xFFu);
+                        int e = 167 - ex;
+                        e = e < 22 ? 22 : (e > 127 ? 127 : e);
+                        pe = __uint_as_float((uint32_t)(e + 127) << 23);
+                        kpow = __uint_as_float((uint32_t)(149 - e + 127) << 23);
+                        neg_bias = -65536.0f * usum;
+                    }
+                    if (!w4::mbar_wait(&tfull[b], (uint32_t)(kbg / NTB) & 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // dx_b * 2^e (exact power-of-two scaling); 0 for rows past M
+                    const float sc = t_live ? __ldg(dx_row + g * 8 + (kb & 7)) * pe : 0.0f;
+                    // two 32-column halves; the buffer is released after the second
+                    // load has landed in registers
+                    const uint32_t ta = tm_row + (uint32_t)(b * BN);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t r[32];
+                        tmem_ld32(ta + 32 * hh, r);
+                        tmem_wait_ld();
+                        if (hh == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) w4::mbar_arrive(&tempty[b]);
+                        }
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            acc[32 * hh + c] = fmaf(sc, __uint_as_float(r[c]), acc[32 * hh + c]);
+                    }
+                    if ((kb & 7) == 7) {
+                        // y += d * (acc * 2^(149-e) - 65536 * sum dx) + m * sum dx S
+                        const float4* dg =
+                            reinterpret_cast<const float4*>(d_s + g * BN + cs * kEpiCols);
+                        const float4* mg =
+                            reinterpret_cast<const float4*>(m_s + g * BN + cs * kEpiCols);
+#pragma unroll
+                        for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                            const float4 dv = dg[c4], mv = mg[c4];
+                            const float dvv[4] = {dv.x, dv.y, dv.z, dv.w};
+                            const float mvv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                            for (int e4 = 0; e4 < 4; ++e4) {
+                                const int c = 4 * c4 + e4;
+                                const float a = fmaf(acc[c], kpow, neg_bias);
+                                yv[c] = fmaf(dvv[e4], a, fmaf(mvv[e4], tmin, yv[c]));
+                                acc[c] = 0.0f;
+                            }
+                        }
+                    }
+                }
+            }
+            // ---- store: directly, or through the split-K workspace ----
+            const int nb = n0 + cs * kEpiCols;
+            bool store = ok && t_live;
+            if (p.splits > 1) {
+                // every epilogue thread reaches both barriers, aborted or not
+                const int tile = tmi * p.tiles_n + tni;
+                const int split = u % p.splits;
+                if (ok) {
+                    float* mine = p.partials +
+                                  (((size_t)tile * p.splits + split) * BM + row) * BN +
+                                  cs * kEpiCols;
+#pragma unroll
+                    for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
+                        *reinterpret_cast<float4*>(mine + 4 * c4) = make_float4(
+                            yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
+                }
+                __threadfence();
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                if (threadIdx.x == 128) {
+                    int last = 0;
+                    if (!*abort_flag) last = atomicAdd(p.counters + tile, 1) == p.splits - 1;
+                    *last_flag = last;
+                }
+                asm volatile("bar.sync 1, 256;" ::: "memory");
+                const bool last = *last_flag != 0;
+                store = store && last;
+                if (last) {
+                    __threadfence();
+                    const float* base =
+                        p.partials + ((size_t)tile * p.splits * BM + row) * BN + cs * kEpiCols;
+#pragma unroll
+                    for (int c = 0; c < kEpiCols; ++c) yv[c] = 0.0f;
+                    for (int q = 0; q < p.splits; ++q) {
+                        const float4* src =
+                            reinterpret_cast<const float4*>(base + (size_t)q * BM * BN);
+#pragma unroll
+                        for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                            const float4 v = __ldcg(src + c4);
+                            yv[4 * c4] += v.x;
+                            yv[4 * c4 + 1] += v.y;
+                            yv[4 * c4 + 2] += v.z;
+                            yv[4 * c4 + 3] += v.w;
+                        }
+                    }
+                    if (threadIdx.x == 128) p.counters[tile] = 0;  // ready for the next call
+                }
+            }
+            if (store) {
+                if (p.out_f32) {
+                    float* yr = reinterpret_cast<float*>(p.y) + (size_t)t * p.N;
+                    if (nb + kEpiCols <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+                        for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
+                            *reinterpret_cast<float4*>(yr + nb + 4 * c4) = make_float4(
+                                yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            dxg[i] = 0.0f;
-                            sg[i] = 0;
-                        }
-                    }
-                    float dmax = 0.0f, usum = 0.0f;
-                    tmin = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        dmax = fmaxf(dmax, dxg[i]);
-                        usum += dxg[i];
-                        tmin = fmaf(dxg[i], (float)sg[i], tmin);
-                    }
-                    // e: dmax * 2^e in [2^40, 2^41), clamped to [22, 127]
-                    const int ex = (int)((__float_as_uint(dmax) >> 23) & 0xFFu);
-                    int e = 167 - ex;
-                    e = e < 22 ? 22 : (e > 127 ? 127 : e);
-                    pe = __uint_as_float((uint32_t)(e + 127) << 23);
-                    kpow = __uint_as_float((uint32_t)(149 - e + 127) << 23);
-                    neg_bias = -65536.0f * usum;
-                }
-                if (!w4::mbar_wait(&tfull[q], (uint32_t)ks & 1u, abort_flag, p.err)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                // dx_b * 2^e (exact power-of-two scaling); 0 for rows past M
-                const float sc = t_live ? __ldg(dx_row + g_begin * 8 + kb) * pe : 0.0f;
-                // two 32-column halves: load, refill with the bias, accumulate
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t r[32];
-                    const uint32_t ta = tm_row + (uint32_t)(q * BN + 32 * hh);
-                    tmem_ld32(ta, r);
-                    tmem_wait_ld();
-                    tmem_fill32(ta, kBias);
-#pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        acc[32 * hh + c] = fmaf(sc, __uint_as_float(r[c]), acc[32 * hh + c]);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) w4::mbar_arrive(&tempty[q]);
-                if ((kb & 7) == 7) {
-                    const int gl = g;  // d_s/m_s hold every group of the row block
-                    const float4* dg = reinterpret_cast<const float4*>(d_s + gl * BN + h * 64);
-                    const float4* mg = reinterpret_cast<const float4*>(m_s + gl * BN + h * 64);
-#pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        const float4 dv = dg[c4], mv = mg[c4];
-                        const float dvv[4] = {dv.x, dv.y, dv.z, dv.w};
-                        const float mvv[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const int c = 4 * c4 + e4;
-                            const float a = fmaf(acc[c], kpow, neg_bias);
-                            yv[c] = fmaf(dvv[e4], a, fmaf(mvv[e4], tmin, yv[c]));
-                            acc[c] = 0.0f;
-                        }
-                    }
-                }
-            }
-        }
-        // ---- store: directly, or through the split-K workspace ----
-        const int nb = n0 + h * 64;
-        bool store = ok && t_live;
-        if (p.splits > 1) {
-            // Every epilogue thread reaches both barriers, aborted or not.
-            const int tile = blockIdx.y * gridDim.x + blockIdx.x;
-            if (ok) {
-                float* mine =
-                    p.partials + (((size_t)tile * p.splits + blockIdx.z) * BM + row) * BN + h * 64;
-#pragma unroll
-                for (int c4 = 0; c4 < 16; ++c4)
-                    *reinterpret_cast<float4*>(mine + 4 * c4) =
-                        make_float4(yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
-            }
-            __threadfence();
-            asm volatile("bar.sync 1, 256;" ::: "memory");
-            volatile int* last_flag = abort_flag + 1;
-            if (threadIdx.x == 128) {
-                int last = 0;
-                if (!*abort_flag) last = atomicAdd(p.counters + tile, 1) == p.splits - 1;
-                *last_flag = last;
-            }
-            asm volatile("bar.sync 1, 256;" ::: "memory");
-            const bool last = *last_flag != 0;
-            store = store && last;
-            if (last) {
-                __threadfence();
-                const float* base =
-                    p.partials + ((size_t)tile * p.splits * BM + row) * BN + h * 64;
-#pragma unroll
-                for (int c = 0; c < 64; ++c) yv[c] = 0.0f;
-                for (int q = 0; q < p.splits; ++q) {
-                    const float4* src = reinterpret_cast<const float4*>(base + (size_t)q * BM * BN);
-#pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        const float4 v = __ldcg(src + c4);
-                        yv[4 * c4] += v.x;
-                        yv[4 * c4 + 1] += v.y;
-                        yv[4 * c4 + 2] += v.z;
-                        yv[4 * c4 + 3] += v.w;
-                    }
-                }
-                if (threadIdx.x == 128) p.counters[tile] = 0;  // ready for the next call
-            }
-        }
-        if (store) {
-            if (p.out_f32) {
-                float* yr = reinterpret_cast<float*>(p.y) + (size_t)t * p.N;
-                if (nb + 64 <= p.N && (p.N & 3) == 0) {
-#pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4)
-                        *reinterpret_cast<float4*>(yr + nb + 4 * c4) =
-                            make_float4(yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (nb + c < p.N) yr[nb + c] = yv[c];
-                }
-            } else {
-                __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)t * p.N;
-                if (nb + 64 <= p.N && (p.N & 7) == 0) {
-#pragma unroll
-                    for (int c8 = 0; c8 < 8; ++c8) {
-                        uint4 v;
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(yv[8 * c8 + 0], yv[8 * c8 + 1]);
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(yv[8 * c8 + 2], yv[8 * c8 + 3]);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(yv[8 * c8 + 4], yv[8 * c8 + 5]);
-                        __nv_bfloat162 h3 = __floats2bfloat162_rn(yv[8 * c8 + 6], yv[8 * c8 + 7]);
-                        v.x = *reinterpret_cast<uint32_t*>(&h0);
-                        v.y = *reinterpret_cast<uint32_t*>(&h1);
-                        v.z = *reinterpret_cast<uint32_t*>(&h2);
-                        v.w = *reinterpret_cast<uint32_t*>(&h3);
-                        *reinterpret_cast<uint4*>(yr + nb + 8 * c8) = v;
+                        for (int c = 0; c < kEpiCols; ++c)
+                            if (nb + c < p.N) yr[nb + c] = yv[c];
                     }
                 } else {
+                    __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)t * p.N;
+                    if (nb + kEpiCols <= p.N && (p.N & 7) == 0) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (nb + c < p.N) yr[nb + c] = __float2bfloat16_rn(yv[c]);
+                        for (int c8 = 0; c8 < kEpiCols / 8; ++c8) {
+                            uint4 v;
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(yv[8 * c8 + 0], yv[8 * c8 + 1]);
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(yv[8 * c8 + 2], yv[8 * c8 + 3]);
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(yv[8 * c8 + 4], yv[8 * c8 + 5]);
+                            __nv_bfloat162 h3 = __floats2bfloat162_rn(yv[8 * c8 + 6], yv[8 * c8 + 7]);
+                            v.x = *reinterpret_cast<uint32_t*>(&h0);
+                            v.y = *reinterpret_cast<uint32_t*>(&h1);
+                            v.z = *reinterpret_cast<uint32_t*>(&h2);
+                            v.w = *reinterpret_cast<uint32_t*>(&h3);
+                            *reinterpret_cast<uint4*>(yr + nb + 8 * c8) = v;
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < kEpiCols; ++c)
+                            if (nb + c < p.N) yr[nb + c] = __float2bfloat16_rn(yv[c]);
+                    }
                 }
             }
         }
@@ -683,7 +728,9 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
         e = cudaMemsetAsync(workspace, 0, (size_t)tiles * 4, (cudaStream_t)stream);
         if (e != cudaSuccess) return w4::cuda_fail(e);
     }
-    dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + BM - 1) / BM), (unsigned)splits);
+    prm.tiles_n = (int)((N + BN - 1) / BN);
+    prm.units = (int)(tiles * splits);
+    const int grid = prm.units < w4::sm_count() ? prm.units : w4::sm_count();
     w4a8_mmq_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, prm);
     return w4::launch_status();
 }
