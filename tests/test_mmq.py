@@ -67,20 +67,28 @@ def test_small_shapes_all_outputs(torch, w4, orc, M, N, K):
     _both(torch, w4, orc, codes, d, m, qa, dx, S, what=f"M{M} N{N} K{K}")
 
 
-def test_extreme_integer_products(torch, w4, orc):
+@pytest.mark.parametrize("scales", ["equal", "varying"])
+def test_extreme_integer_products(torch, w4, orc, scales):
     # all codes 15 and all activations +-127: |P| = 32*15*127 per block, the
-    # largest block dot product the format allows
+    # largest block dot product the format allows; token rows 0-63 reach +P
+    # in every block, rows 64-95 -P in every block (the two ends of the
+    # integer range a 256-group can accumulate), the rest mixed signs.
+    # "varying" draws a different scale for every block.
     M, N, K = 128, 128, 1024
     codes = np.full((N, K // 2), 0xFF, np.uint8)
     d = synth.f32_to_f16_bits(np.full((N, K // 256), 0.01, np.float32))
     m = synth.f32_to_f16_bits(np.full((N, K // 256), -0.05, np.float32))
     sign = np.where(np.random.default_rng(1).random((M, K)) < 0.5, -1, 1)
     sign[:64] = 1
+    sign[64:96] = -1
     qa = (127 * sign).astype(np.int8)
-    dx = np.full((M, K // 32), 0.03, np.float32)
+    if scales == "equal":
+        dx = np.full((M, K // 32), 0.03, np.float32)
+    else:
+        dx = np.random.default_rng(2).uniform(0.001, 0.05, (M, K // 32)).astype(np.float32)
     S = qa.astype(np.int32).reshape(M, K // 32, 32).sum(axis=2).astype(np.int32)
-    P = orc.mmq_blockdots(codes[:1], qa[:1])
-    assert P.max() == 32 * 15 * 127
+    P = orc.mmq_blockdots(codes[:1], qa)
+    assert P.max() == 32 * 15 * 127 and P.min() == -32 * 15 * 127
     _both(torch, w4, orc, codes, d, m, qa, dx, S, what="extreme")
 
 

@@ -12,41 +12,50 @@
 // Persistent CTAs (one per SM) loop over work units = (128-token x 128-row
 // output tile, K slice); the pipeline, barriers and TMEM allocation live for
 // the whole launch.  K advances in stages of 128 (four 32-element activation
-// blocks):
+// blocks); two stages make one 256-group.
 //   warp 0      TMA producer: the qa tile (128 x 128 B, 128B-swizzled) and the
 //               packed code tile (128 rows x 64 B) into a 4-stage ring.
-//   warp 1      allocates 512 TMEM columns; one lane issues, per 32-block, one
-//               tcgen05.mma.kind::i8 (M=128, N=128, K=32; A = qa as s8, B = the
-//               codes as u8) into its own 128-column TMEM buffer, so every
-//               block's exact int32 products stay separate.
+//   warp 1      allocates 512 TMEM columns = four 128-column block buffers;
+//               one lane issues, per 32-block, a tcgen05.mma.kind::i8 (M=128,
+//               N=128, K=32; A = qa as s8, B = the codes as u8) into the
+//               buffer of the block's position in the stage, and one
+//               tcgen05.commit per buffer pair.
 //   warps 2-3   unpack each code tile, nibble -> byte, into the 128B-swizzled
 //               K-major layout the MMA's shared-memory descriptor expects
 //               (tcgen05 has no 4-bit integer kind).
 //   warps 4-11  epilogue: each thread owns one token row (its TMEM lane) and 64
-//               weight rows.  Per block it loads its 64 words with one wait,
-//               refills the bias and releases the buffer before any arithmetic,
-//               so the MMA only waits on TMEM round trips, not on the FMAs.
+//               weight rows; per buffer pair it waits once, reads both blocks'
+//               words and releases the pair; the thread that sees a stage's
+//               last pair also frees that stage's shared-memory operands.
+//
+// On B200 the tensor pipe runs MMAs and commits one after another, and a
+// commit costs about as much as 1.5 of these MMAs (measured), so commits are
+// per pair of blocks rather than per block, and the shared-memory stage is
+// released by the epilogue, not by a further commit.
 //
 // Epilogue arithmetic.  Converting 16384 int32 products per block to float at
 // the quarter-rate conversion throughput would cost four times the MMA, so
-// no conversion is done: before each block's MMA the tensor core writes the
-// integer bias 65536 into the block's TMEM buffer (a second kind::i8 MMA over
-// constant u8 tiles, 32 * 32 * 64 = 65536, in overwrite mode), and the block's
-// MMA accumulates onto it (|P| <= 32*15*127 = 60960), so the word read back
-// is V = 65536 + P in [4576, 126496] -- as fp32 bits, the exact denormal
-// V * 2^-149.  With dx scaled by a power of two 2^e chosen per (token, group)
-// so that products stay normal, one full-rate FMA per element accumulates
-// acc = sum_b (dx_b 2^e) V_b 2^-149, and at the group end
-//   sum_b dx_b P_b = acc * 2^(149-e) - 65536 * sum_b dx_b
-// (one FMA, a single rounding), then y += d * that + m * sum_b dx_b S_b.
-// The TMEM-to-register path (about 340 B per SM per clock on B200, measured)
-// is what bounds this kernel: every block's 128 x 128 int32 products must be
-// read once.  Requires |dx| < 2^100 (activations far beyond any fp16/bf16
-// model range would overflow the scaled products).
+// no conversion is done.  At the start of each 256-group the tensor core
+// seeds every buffer with the integer 2^17 (a kind::i8 MMA over constant u8
+// tiles, 32 * 64 * 64, in overwrite mode); buffer r then accumulates block r
+// of the group and, in the second stage, block r + 4 on top of it.  With
+// |P| <= 32*15*127 = 60960 per block, the words read back,
+//   V_r = 2^17 + P_r   and   V_{r+4} = 2^17 + P_r + P_{r+4},
+// lie in [9152, 252992] -- as fp32 bits, exact denormals V * 2^-149.  Abel
+// summation turns the per-block scaling into one full-rate FMA per element
+// per block with per-(token, block) coefficients:
+//   sum_b dx_b P_b = sum_{r<4} [ (dx_r - dx_{r+4}) V_r + dx_{r+4} V_{r+4} ]
+//                    - 2^17 sum_{r<4} dx_r,
+// the coefficients scaled by a power of two 2^e per (token, group) so that
+// the products stay normal.  At the group end one FMA recovers
+// acc * 2^(149-e) - 2^17 sum_{r<4} dx_r, and y += d * that + m * sum_b dx_b S_b.
+// The exact integer block sums never leave TMEM as anything but exact values;
+// the fp32 work is the coefficient differences and the accumulation.
+// Requires |dx| < 2^100 (activations far beyond any fp16/bf16 model range
+// would overflow the scaled products).
 //
-// The MMA runs up to four blocks ahead of the epilogue (four TMEM buffers).
-// Registers are rebalanced with setmaxnreg: 72 per thread for warps 0-3, 216
-// for the epilogue (128*72 + 256*216 = 384*168, the launch allotment).
+// Registers are rebalanced with setmaxnreg: 40 per thread for warps 0-3, 232
+// for the epilogue (128*40 + 256*232 = 384*168, the launch allotment).
 // K slices (split-K) write fp32 partial tiles to the caller's workspace; the
 // CTA that finishes a tile last sums the partials in slice order (bitwise
 // deterministic) and stores y.
@@ -68,9 +77,10 @@ constexpr int BN = 128;        // weight rows per tile (MMA N)
 constexpr int BK = 128;        // K elements per pipeline stage
 constexpr int KB = 32;         // activation block = MMA K for kind::i8
 constexpr int STAGES = 4;
-constexpr int NBLK = BK / KB;  // 32-blocks per pipeline stage
 constexpr int NTB = 4;         // TMEM block buffers (BN columns each)
+constexpr int NPAIR = NTB / 2; // buffer pairs: the unit of MMA -> epilogue hand-off
 constexpr int BIAS_BYTES = 128 * KB;  // one constant operand tile of the bias MMA
+constexpr int kBiasLog2 = 17;         // accumulator bias 2^17 (see the header)
 constexpr int kThreads = 384;              // 4 producer-side warps + 8 epilogue warps
 constexpr int kEpiWarps = 8;
 constexpr int kEpiCols = BN / (kEpiWarps / 4); // 64 weight rows per epilogue thread
@@ -88,7 +98,7 @@ struct Smem {
     static constexpr int bp = b + STAGES * B_BYTES;
     static constexpr int bias = bp + STAGES * BP_BYTES;  // bias MMA operands (A, B)
     static constexpr int bars = bias + 2 * BIAS_BYTES;   // uint64 barriers
-    static constexpr int nbars = 3 * STAGES + 2 * NTB + 1;
+    static constexpr int nbars = 3 * STAGES + 2 * NPAIR + 1;
     static constexpr int misc = bars + nbars * 8;        // tmem base, abort flag
     static constexpr int dm = (misc + 16 + 15) & ~15;    // fp32 d[G][BN], m[G][BN]
     static size_t total(int G) { return (size_t)dm + (size_t)2 * G * BN * 4 + 1024; }
@@ -189,10 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bars);
     uint64_t* full = bars;                   // TMA landed (A + packed B)
     uint64_t* unpacked = bars + STAGES;      // B unpacked into the MMA layout
-    uint64_t* empty = bars + 2 * STAGES;     // MMAs of the stage done
-    uint64_t* tfull = bars + 3 * STAGES;     // TMEM buffer written
-    uint64_t* tempty = tfull + NTB;          // TMEM buffer drained and refilled
-    uint64_t* drain = tempty + NTB;          // final MMA completion
+    uint64_t* empty = bars + 2 * STAGES;     // MMAs of the stage done (seen by the epilogue)
+    uint64_t* tfull = bars + 3 * STAGES;     // TMEM buffer pair written
+    uint64_t* tempty = tfull + NPAIR;        // TMEM buffer pair read out
+    uint64_t* drain = tempty + NPAIR;        // final MMA completion
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Smem::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
     volatile int* last_flag = abort_flag + 1;
@@ -221,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             w4::mbar_init(&unpacked[i], 2);
             w4::mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < NTB; ++i) {
+        for (int i = 0; i < NPAIR; ++i) {
             w4::mbar_init(&tfull[i], 1);
             w4::mbar_init(&tempty[i], kEpiWarps);
         }
@@ -229,12 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         w4::fence_mbar_init();
     }
-    // constant operands of the bias MMA: A = 32, B = 64 (u8), so that over K = 32
-    // every accumulator starts at 32 * 32 * 64 = 65536
+    // constant operands of the bias MMA: A = B = 64 (u8), so that over K = 32
+    // every accumulator starts at 32 * 64 * 64 = 2^17
     {
         uint32_t* ba = reinterpret_cast<uint32_t*>(smem + Smem::bias);
         for (int i = threadIdx.x; i < 2 * BIAS_BYTES / 4; i += kThreads)
-            ba[i] = i < BIAS_BYTES / 4 ? 0x20202020u : 0x40404040u;
+            ba[i] = 0x40404040u;
         w4::fence_proxy_async_smem();
     }
     if (warp == 1) {
@@ -250,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
         if (warp == 0) {
             // ---------------- TMA producer ----------------
             if (w4::elect_one()) {
@@ -308,24 +318,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         const uint32_t a_addr = w4::smem_u32(sa + s * A_BYTES);
                         const uint32_t b_addr = w4::smem_u32(sb + s * B_BYTES);
-                        for (int q = 0; q < NBLK; ++q) {
-                            // block kbg goes to buffer kbg % NTB; wait until the epilogue
-                            // has read that buffer's previous block (first use: free)
-                            const int kbg = it * NBLK + q;
-                            const int b = kbg % NTB;
-                            const uint32_t par = ((uint32_t)(kbg / NTB) & 1u) ^ 1u;
-                            if (!w4::mbar_wait(&tempty[b], par, abort_flag, p.err)) {
+                        // First half of a 256-group (stage kg even): each buffer is
+                        // seeded with the bias before its block; second half: the
+                        // block accumulates onto the first half's block in that buffer.
+                        const bool seed = (kg & 1) == 0;
+                        for (int j = 0; j < NPAIR && ok; ++j) {
+                            // wait until the epilogue has read this pair's previous
+                            // blocks (first use: free)
+                            if (!w4::mbar_wait(&tempty[j], ((uint32_t)it & 1u) ^ 1u, abort_flag,
+                                               p.err)) {
                                 ok = false;
                                 break;
                             }
                             tc_fence_after();
-                            const uint32_t dt = tmem_base + (uint32_t)(b * BN);
-                            mma_i8(dt, bias_a, bias_b, idesc_bias, 0u);  // D = 65536
-                            mma_i8(dt, smem_desc_sw128(a_addr + q * KB),
-                                   smem_desc_sw128(b_addr + q * KB), idesc, 1u);  // D += P
-                            mma_commit(&tfull[b]);
+#pragma unroll
+                            for (int qq = 0; qq < 2; ++qq) {
+                                const int q = 2 * j + qq;  // block in the stage = buffer
+                                const uint32_t dt = tmem_base + (uint32_t)(q * BN);
+                                if (seed) mma_i8(dt, bias_a, bias_b, idesc_bias, 0u);  // D = 2^17
+                                mma_i8(dt, smem_desc_sw128(a_addr + q * KB),
+                                       smem_desc_sw128(b_addr + q * KB), idesc, 1u);  // D += P
+                            }
+                            mma_commit(&tfull[j]);
                         }
-                        mma_commit(&empty[s]);
                     }
                 }
                 mma_commit(drain);
@@ -371,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue (warps 4..11) ----------------
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
         const int et = threadIdx.x - 128;           // 0..255
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
         const int cs = (warp - 4) >> 2;             // column slice: kEpiCols weight rows
@@ -409,84 +424,105 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc[c] = 0.0f;
                 yv[c] = 0.0f;
             }
-            float pe = 0.0f, kpow = 0.0f, neg_bias = 0.0f, tmin = 0.0f;
+            float kpow = 0.0f, neg_bias = 0.0f, tmin = 0.0f;
+            float cf[8];  // per-block coefficients of the current group, times 2^e
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cf[i] = 0.0f;
             const float* dx_row = p.dx + (size_t)(t_live ? t : 0) * B;
+            const int32_t* s_row = p.S + (size_t)(t_live ? t : 0) * B;
             const int ksteps = (g_end - g_begin) * 2;
             for (int ks = 0; ks < ksteps && ok; ++ks, ++it) {
-#pragma unroll 1
-                for (int q = 0; q < NBLK; ++q) {
-                    const int kb = ks * NBLK + q;         // block index within the slice
-                    const int kbg = it * NBLK + q;        // global block counter
-                    const int b = kbg % NTB;              // its TMEM buffer
-                    const int g = g_begin + (kb >> 3);    // global group index
-                    if ((kb & 7) == 0) {
-                        // group set-up: max, sum and S-weighted sum of the 8 block scales
-                        float dmax = 0.0f, usum = 0.0f;
-                        tmin = 0.0f;
-                        if (t_live) {
+                const int g = g_begin + (ks >> 1);  // global group index
+                const bool first_half = (ks & 1) == 0;
+                if (first_half) {
+                    // group set-up from the 8 block scales dx_0..dx_7 of this token:
+                    // buffer r holds V_r = 2^17 + P_r after block r and
+                    // V_{r+4} = 2^17 + P_r + P_{r+4} after block r + 4, so
+                    //   sum_b dx_b P_b = sum_{r<4} (dx_r - dx_{r+4}) V_r + dx_{r+4} V_{r+4}
+                    //                    - 2^17 sum_{r<4} dx_r
+                    float dxg[8];
 #pragma unroll
-                            for (int h4 = 0; h4 < 2; ++h4) {
-                                const float4 a = __ldg(reinterpret_cast<const float4*>(dx_row + g * 8) + h4);
-                                const int4 sv =
-                                    __ldg(reinterpret_cast<const int4*>(p.S + (size_t)t * B + g * 8) + h4);
-                                dmax = fmaxf(fmaxf(dmax, fmaxf(a.x, a.y)), fmaxf(a.z, a.w));
-                                usum += a.x; usum += a.y; usum += a.z; usum += a.w;
-                                tmin = fmaf(a.x, (float)sv.x, tmin);
-                                tmin = fmaf(a.y, (float)sv.y, tmin);
-                                tmin = fmaf(a.z, (float)sv.z, tmin);
-                                tmin = fmaf(a.w, (float)sv.w, tmin);
-                            }
+                    for (int i = 0; i < 8; ++i) dxg[i] = 0.0f;
+                    tmin = 0.0f;
+                    if (t_live) {
+#pragma unroll
+                        for (int h4 = 0; h4 < 2; ++h4) {
+                            const float4 a = __ldg(reinterpret_cast<const float4*>(dx_row + g * 8) + h4);
+                            const int4 sv = __ldg(reinterpret_cast<const int4*>(s_row + g * 8) + h4);
+                            dxg[4 * h4] = a.x;
+                            dxg[4 * h4 + 1] = a.y;
+                            dxg[4 * h4 + 2] = a.z;
+                            dxg[4 * h4 + 3] = a.w;
+                            tmin = fmaf(a.x, (float)sv.x, tmin);
+                            tmin = fmaf(a.y, (float)sv.y, tmin);
+                            tmin = fmaf(a.z, (float)sv.z, tmin);
+                            tmin = fmaf(a.w, (float)sv.w, tmin);
                         }
-                        // e: dmax * 2^e in [2^40, 2^41), clamped to [22, 127]
-                        const int ex = (int)((__float_as_uint(dmax) >> 23) & 0xFFu);
-                        int e = 167 - ex;
-                        e = e < 22 ? 22 : (e > 127 ? 127 : e);
-                        pe = __uint_as_float((uint32_t)(e + 127) << 23);
-                        kpow = __uint_as_float((uint32_t)(149 - e + 127) << 23);
-                        neg_bias = -65536.0f * usum;
                     }
-                    if (!w4::mbar_wait(&tfull[b], (uint32_t)(kbg / NTB) & 1u, abort_flag, p.err)) {
+                    float dmax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) dmax = fmaxf(dmax, dxg[i]);
+                    // e: dmax * 2^e in [2^40, 2^41), clamped to [22, 127]
+                    const int ex = (int)((__float_as_uint(dmax) >> 23) & 0xFFu);
+                    int e = 167 - ex;
+                    e = e < 22 ? 22 : (e > 127 ? 127 : e);
+                    const float pe = __uint_as_float((uint32_t)(e + 127) << 23);
+                    kpow = __uint_as_float((uint32_t)(149 - e + 127) << 23);
+                    neg_bias = -(float)(1 << kBiasLog2) * ((dxg[0] + dxg[1]) + (dxg[2] + dxg[3]));
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        cf[r] = (dxg[r] - dxg[r + 4]) * pe;
+                        cf[r + 4] = dxg[r + 4] * pe;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < NPAIR; ++j) {
+                    if (!ok) break;
+                    if (!w4::mbar_wait(&tfull[j], (uint32_t)it & 1u, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    // dx_b * 2^e (exact power-of-two scaling); 0 for rows past M
-                    const float sc = t_live ? __ldg(dx_row + g * 8 + (kb & 7)) * pe : 0.0f;
-                    // two 32-column halves; the buffer is released after the second
-                    // load has landed in registers
-                    const uint32_t ta = tm_row + (uint32_t)(b * BN);
+                    // the stage's last pair has landed: its shared-memory operands are free
+                    if (j == NPAIR - 1 && threadIdx.x == 128) w4::mbar_arrive(&empty[it % STAGES]);
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        uint32_t r[32];
-                        tmem_ld32(ta + 32 * hh, r);
-                        tmem_wait_ld();
-                        if (hh == 1) {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) w4::mbar_arrive(&tempty[b]);
-                        }
+                    for (int qq = 0; qq < 2; ++qq) {
+                        const int q = 2 * j + qq;  // block in the stage = buffer
+                        const float sc = first_half ? cf[q] : cf[q + 4];
+                        const uint32_t ta = tm_row + (uint32_t)(q * BN);
+                        // two 32-column halves; the pair is released once the
+                        // second block's words are in registers
 #pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            acc[32 * hh + c] = fmaf(sc, __uint_as_float(r[c]), acc[32 * hh + c]);
-                    }
-                    if ((kb & 7) == 7) {
-                        // y += d * (acc * 2^(149-e) - 65536 * sum dx) + m * sum dx S
-                        const float4* dg =
-                            reinterpret_cast<const float4*>(d_s + g * BN + cs * kEpiCols);
-                        const float4* mg =
-                            reinterpret_cast<const float4*>(m_s + g * BN + cs * kEpiCols);
-#pragma unroll
-                        for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
-                            const float4 dv = dg[c4], mv = mg[c4];
-                            const float dvv[4] = {dv.x, dv.y, dv.z, dv.w};
-                            const float mvv[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-                            for (int e4 = 0; e4 < 4; ++e4) {
-                                const int c = 4 * c4 + e4;
-                                const float a = fmaf(acc[c], kpow, neg_bias);
-                                yv[c] = fmaf(dvv[e4], a, fmaf(mvv[e4], tmin, yv[c]));
-                                acc[c] = 0.0f;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            uint32_t r[32];
+                            tmem_ld32(ta + 32 * hh, r);
+                            tmem_wait_ld();
+                            if (qq == 1 && hh == 1) {
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) w4::mbar_arrive(&tempty[j]);
                             }
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                acc[32 * hh + c] = fmaf(sc, __uint_as_float(r[c]), acc[32 * hh + c]);
+                        }
+                    }
+                }
+                if (ok && !first_half) {
+                    // y += d * (acc * 2^(149-e) - 2^17 * sum_{r<4} dx_r) + m * sum dx S
+                    const float4* dg = reinterpret_cast<const float4*>(d_s + g * BN + cs * kEpiCols);
+                    const float4* mg = reinterpret_cast<const float4*>(m_s + g * BN + cs * kEpiCols);
+#pragma unroll
+                    for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                        const float4 dv = dg[c4], mv = mg[c4];
+                        const float dvv[4] = {dv.x, dv.y, dv.z, dv.w};
+                        const float mvv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const int c = 4 * c4 + e4;
+                            const float av = fmaf(acc[c], kpow, neg_bias);
+                            yv[c] = fmaf(dvv[e4], av, fmaf(mvv[e4], tmin, yv[c]));
+                            acc[c] = 0.0f;
                         }
                     }
                 }
