@@ -294,6 +294,33 @@ def time_gemv_sweep(torch, w4, wl, M, steps, warmup, stream):
     return elapsed, per, steps * len(SHAPES)
 
 
+def time_gemv_back_to_back(torch, w4, wl, s, reps, stream):
+    """Steady-state duration of one shape's GEMV: `reps` launches in one CUDA
+    graph, consecutive launches on alternating weight copies, event-timed on
+    the launching stream; ms per launch.  Only meaningful for shapes whose
+    two weight copies exceed L2 (every launch then streams from HBM)."""
+    xs, ys = wl.xs(1)
+    ncopy = len(wl.weights)
+
+    def burst():
+        for i in range(reps):
+            codes, d, m = wl.weights[i % ncopy][s]
+            w4.w4_gemv(codes, d, m, xs[s], out_dtype=torch.bfloat16, y=ys[s], stream=stream)
+
+    g = _capture(torch, stream, burst)
+    with torch.cuda.stream(stream):
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / (3 * reps)
+
+
 def time_e2e(torch, w4, wl, steps, warmup, stream):
     """Same sweep through host buffers: pinned x -> device, GEMVs, y -> host."""
     M = 1
@@ -458,15 +485,22 @@ def run_ours(args):
     elapsed_max, bytes_all = reduce_timing(elapsed, step_bytes * args.steps, dev)
     value = bytes_all / elapsed_max / 1e9
 
-    # dominant kernel: the lm_head GEMV (largest stream, ~80% of the step)
+    # dominant kernel: the lm_head GEMV (largest stream, ~80% of the step);
+    # its duration back to back (steady state, both weight copies > L2), and
+    # the isolated single launch (launch ramp included) for reference
     N, K = SHAPES[4]
     dom_bytes = gemv_bytes(N, K, 1)
-    dom_s = per_shape_ms[4] / 1e3
+    dom_ms = time_gemv_back_to_back(torch, w4, wl, 4, 8, stream)
+    dom_s = dom_ms / 1e3
     achieved = dom_bytes / dom_s / 1e9
+    isolated = dom_bytes / (per_shape_ms[4] / 1e3) / 1e9
     traffic = load_traffic("w4_quant_matmul_b200/csrc/gemv.cu", "w4_gemv_lm_head_m1")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic, "kernel": "w4_gemv_kernel (151936x2560, M=1)",
+                "traffic": traffic, "kernel": "w4_gemv_rows_kernel (151936x2560, M=1)",
+                "duration_us": round(dom_ms * 1e3, 2),
+                "timing": "8 back-to-back launches per CUDA graph, alternating 200 MB weight copies",
+                "isolated_achieved": round(isolated, 1),
                 "algorithmic_bytes": dom_bytes,
                 "peak_source": f"{peaks['source']} hbm_gbs"}
 

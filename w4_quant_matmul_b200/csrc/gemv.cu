@@ -23,22 +23,34 @@
 //    4 dp4a per token, and sum_k q X is exact: 256 * sum(q Xh) + sum(q Xl)
 //    (|.| <= 32 * 15 * 32640 < 2^24, exact in fp32 too).  Per chunk
 //        sum q x ~= (sum q X) / sigma,    y += d * that + m * Sx.
-//  * Work split.  A half-warp (16 lanes) owns RH rows and one of KS K-slices;
-//    lane j streams the 16-byte code chunks (32 codes) c = j, j+16, ... of its
-//    slice with non-allocating 128-bit loads, U chunks ahead per row.  With
-//    KS > 1 the slices of a row are summed in fixed order through shared
-//    memory (small-N shapes need the extra streams); with KS = 1 a 4-step
-//    xor-shuffle finishes the row.  CTAs loop over row blocks.  The staged
-//    activation words are chunk-minor ([word][chunk]) so the 16 lanes of a
-//    half-warp read 16 different banks.
-//  * Programmatic dependent launch.  Before griddepcontrol.wait the CTA only
-//    asks L2 to prefetch its first batch of weights (bulk L2 prefetch; L2 is
+//
+// Two ways of feeding that inner loop, chosen by the size of the weight stream:
+//
+//  * Row kernel (large streams, e.g. the lm_head).  A half-warp (16 lanes)
+//    owns RH rows and one of KS K-slices; lane j streams the 16-byte code
+//    chunks c = j, j+16, ... of its slice with non-allocating 128-bit loads, U
+//    chunks ahead per row, and each activation word it reads serves RH rows.
+//    With KS > 1 the slices of a row are summed in fixed order through shared
+//    memory; with KS = 1 a 4-step xor-shuffle finishes the row.  CTAs loop
+//    over row blocks.
+//  * Ring kernel (streams below 16 MB, where a few latency-bound rounds of the
+//    row kernel and their imbalance dominate).  Every CTA gets one contiguous
+//    range of rows of equal length; a producer lane streams it with bulk TMA
+//    copies (cp.async.bulk, 16 rows x a 1280-byte K-chunk per stage) through a
+//    4-stage shared-memory ring completed on mbarriers, so the whole range is
+//    in flight without registers; 16 consumer half-warps run the same inner
+//    loop, one row each, from shared memory.
+//  * Programmatic dependent launch (ring kernel).  Before griddepcontrol.wait
+//    a CTA only asks L2 to prefetch its first weights (bulk L2 prefetch; L2 is
 //    the point of coherence, so a prefetch can never observe stale data even
 //    if the preceding kernel writes the weights).  In a chain of launches the
 //    first HBM round trip of this GEMV overlaps the tail of the previous
-//    kernel; every load that feeds arithmetic happens after the wait.
+//    kernel; every load that feeds arithmetic happens after the wait.  The
+//    row kernel is launched in plain stream order (its dependency wait is
+//    then a no-op): measured in a five-GEMV decode step, its CTAs launched
+//    early behind a ring kernel cost more than the overlap gained.
 // Integer sums are exact and the float reductions run in a fixed order:
-// results are bitwise deterministic.
+// results are bitwise deterministic (for a given shape, which fixes the kernel).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -221,10 +233,10 @@ struct MinCtas {
 };
 
 template <int M, int RH, int U>
-__global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_kernel(
+__global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
     int N, int K, int KS, const uint16_t* __restrict__ x, void* __restrict__ y, int out_f32) {
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(128) unsigned char smem[];
     const int C = K >> 5;  // 32-code chunks per row
     const int G = K >> 8;  // groups per row
     uint4* xq = reinterpret_cast<uint4*>(smem);                                // [M][4][C]
@@ -368,10 +380,10 @@ size_t smem_bytes(int M, int C, int KS, int RH) {
 }
 
 template <int M, int RH>
-int launch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K, int KS,
+int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K, int KS,
            const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
     constexpr int U = 8 / RH;
-    auto kern = w4_gemv_kernel<M, RH, U>;
+    auto kern = w4_gemv_rows_kernel<M, RH, U>;
     const int C = K / 32;
     const size_t smem = smem_bytes(M, C, KS, RH);
     // Per-instantiation cache: one device, a few shared-memory sizes.
@@ -408,16 +420,16 @@ int launch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, in
     int grid = per_sm * w4::sm_count();
     if (grid > nblocks) grid = nblocks;
 
+    // Plain stream order, no programmatic dependent launch: launched early
+    // behind a ring-kernel GEMV, this kernel's resident-but-waiting CTAs cost
+    // ~10 us per five-GEMV decode step (measured), more than the overlap gains.
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
     e = cudaLaunchKernelEx(&cfg, kern, codes, reinterpret_cast<const __half*>(d),
                            reinterpret_cast<const __half*>(m), N, K, KS, x, y, out_f32);
     if (e != cudaSuccess) return w4::cuda_fail(e);
@@ -444,10 +456,324 @@ int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N
     if (M >= 4 && rh > 2) rh = 2;  // register budget: M * RH accumulators twice
     if (smem_bytes(M, K / 32, ks, rh) > (size_t)kSmemBudget) ks = 1;
     if constexpr (M < 4) {
-        if (rh == 4) return launch<M, 4>(codes, d, m, N, K, ks, x, y, out_f32, st);
+        if (rh == 4) return launch_rows<M, 4>(codes, d, m, N, K, ks, x, y, out_f32, st);
     }
-    if (rh >= 2) return launch<M, 2>(codes, d, m, N, K, ks, x, y, out_f32, st);
-    return launch<M, 1>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    if (rh >= 2) return launch_rows<M, 2>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    return launch_rows<M, 1>(codes, d, m, N, K, ks, x, y, out_f32, st);
+}
+
+// ---------------------------------------------------------------------------
+// ring kernel
+// ---------------------------------------------------------------------------
+
+constexpr int kRingWarps = 8;                           // consumers: 16 half-warps, one row each
+constexpr int kRingThreads = 32 * (kRingWarps + 1);     // + the producer warp
+constexpr int kRowsPerStage = 2 * kRingWarps;           // 16
+constexpr int kChunkBytes = 1280;                       // K-chunk of a row per stage
+constexpr int kStageBytes = kRowsPerStage * kChunkBytes;  // 20 KB
+constexpr int kMaxStages = 4;
+constexpr int kSmemPerSm = 227 * 1024;                  // usable per CTA on sm_100
+constexpr size_t kRingMaxCodeBytes = (size_t)16 << 20;  // streams below this use the ring
+
+// Shared memory: [stages][16 rows][1280 B] code ring, then the activation
+// words xq[M][4][C] (uint4), chunk sums sx[M][C], 1/sigma inv[M][C], and the
+// ring's barriers.
+struct Layout {
+    size_t xq, sx, inv, bars, total;
+};
+
+__host__ __device__ inline Layout layout(int M, int C, int stages) {
+    Layout l;
+    l.xq = (size_t)stages * kStageBytes;
+    l.sx = l.xq + (size_t)M * 4 * C * 16;
+    l.inv = l.sx + (size_t)M * C * 4;
+    l.bars = (l.inv + (size_t)M * C * 4 + 7) & ~(size_t)7;
+    l.total = l.bars + 2 * kMaxStages * 8 + 16;
+    return l;
+}
+
+// Resident CTAs per SM the register allocation is sized for (two while the
+// per-token accumulators leave room, so that two rings stream per SM).
+template <int M>
+struct RingMinCtas {
+    static constexpr int value = M <= 4 ? 2 : 1;
+};
+
+template <int M>
+__global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_ring_kernel(
+    const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
+    int N, int K, int stages, int rows_per_cta, const uint16_t* __restrict__ x,
+    void* __restrict__ y, int out_f32, int* err) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int C = K >> 5;          // 32-code chunks per row
+    const int G = K >> 8;          // groups per row
+    const int row_bytes = K >> 1;
+    const int nkc = (row_bytes + kChunkBytes - 1) / kChunkBytes;  // K-chunks per row
+    const Layout L = layout(M, C, stages);
+    uint4* xq = reinterpret_cast<uint4*>(smem + L.xq);
+    float* sx = reinterpret_cast<float*>(smem + L.sx);
+    float* inv = reinterpret_cast<float*>(smem + L.inv);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+    uint64_t* empty = full + kMaxStages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kMaxStages);
+
+    const int warp = threadIdx.x >> 5;
+    const int r0 = blockIdx.x * rows_per_cta;
+    const int r1 = min(N, r0 + rows_per_cta);
+    const int ngrp = (r1 - r0 + kRowsPerStage - 1) / kRowsPerStage;
+    const int nstage = ngrp * nkc;  // stages of this CTA, in (row group, K-chunk) order
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kMaxStages; ++i) {
+            w4::mbar_init(&full[i], 1);
+            w4::mbar_init(&empty[i], kRingWarps);
+        }
+        *abort_flag = 0;
+        w4::fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == kRingWarps) {
+        // ---------------- producer: one lane streams the code ring ----------------
+        if (w4::elect_one()) {
+            // before the dependency wait only L2 prefetches (L2 is the point of
+            // coherence: a prefetch cannot hand stale weights to a later load)
+            const int first = min(kRowsPerStage, r1 - r0);
+            const uint32_t b0 = (uint32_t)min(kChunkBytes, row_bytes);
+            for (int r = 0; r < first; ++r)
+                l2_prefetch(codes + (size_t)(r0 + r) * row_bytes, b0);
+            pdl_wait();
+            int it = 0;
+            for (; it < nstage; ++it) {
+                const int s = it % stages;
+                const uint32_t ph = (uint32_t)(it / stages) & 1u;
+                if (!w4::mbar_wait(&empty[s], ph ^ 1u, abort_flag, err)) break;
+                const int grp = it / nkc, kc = it - grp * nkc;
+                const int rb = r0 + grp * kRowsPerStage;
+                const int nr = min(kRowsPerStage, r1 - rb);
+                const int off = kc * kChunkBytes;
+                const uint32_t bytes = (uint32_t)min(kChunkBytes, row_bytes - off);
+                uint8_t* dst = smem + (size_t)s * kStageBytes;
+                w4::mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)nr);
+                for (int r = 0; r < nr; ++r)
+                    w4::bulk_load_1d(dst + r * kChunkBytes, codes + (size_t)(rb + r) * row_bytes + off,
+                                     bytes, &full[s]);
+            }
+            // every issued copy lands before the CTA may exit
+            for (int k = it - stages < 0 ? 0 : it - stages; k < it; ++k)
+                w4::mbar_wait(&full[k % stages], (uint32_t)(k / stages) & 1u, nullptr, err);
+        }
+        return;
+    }
+
+    // ---------------- consumers (warps 0..7) ----------------
+    const int h = threadIdx.x >> 4;  // half-warp = row slot of a stage
+    const int j = threadIdx.x & 15;  // lane in the half-warp
+    pdl_wait();
+
+    // activation words, chunk sums and scales, once per CTA; each thread issues
+    // up to four 16-byte loads before converting any
+    const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
+    constexpr int kCons = 32 * kRingWarps;
+    for (int base = 0; base < nq; base += 4 * kCons) {
+        uint4 raw[4];
+#pragma unroll
+        for (int p4 = 0; p4 < 4; ++p4) {
+            const int v = base + p4 * kCons + threadIdx.x;
+            raw[p4] = v < nq ? __ldg(reinterpret_cast<const uint4*>(x) + v) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int p4 = 0; p4 < 4; ++p4) {
+            if (base + p4 * kCons >= nq) break;  // uniform across the consumers
+            const int v = base + p4 * kCons + threadIdx.x;
+            const bool live = v < nq;
+            const int vv = live ? v : 0;
+            const int t = vv / (C * 4);
+            const int r = vv - t * C * 4;
+            const int c = r >> 2, q4 = r & 3;
+            stage_quarter(raw[p4], live, &xq[((size_t)t * 4 + q4) * C + c], &sx[t * C + c],
+                          &inv[t * C + c], q4);
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
+    pdl_launch_dependents();
+
+    // d and m of this lane's chunks in a stage: chunk cl = j + 16 i of K-chunk
+    // kc lies in group kc * 10 + 2 i + (j >> 3); loaded one stage ahead
+    constexpr int kLaneChunks = kChunkBytes / 16 / 16;  // 5
+    auto load_dm = [&](int st, uint32_t (&dm)[kLaneChunks]) {
+#pragma unroll
+        for (int i = 0; i < kLaneChunks; ++i) dm[i] = 0;
+        if (st >= nstage) return;
+        const int grp = st / nkc, kc = st - grp * nkc;
+        const int row = r0 + grp * kRowsPerStage + h;
+        if (row >= r1) return;
+        const int nch = min(kChunkBytes, row_bytes - kc * kChunkBytes) >> 4;
+#pragma unroll
+        for (int i = 0; i < kLaneChunks; ++i) {
+            if (j + 16 * i < nch) {
+                const size_t gi = (size_t)row * G + kc * (kChunkBytes / 128) + 2 * i + (j >> 3);
+                dm[i] = (uint32_t)ld_nc_u16(d + gi) | ((uint32_t)ld_nc_u16(m + gi) << 16);
+            }
+        }
+    };
+
+    // d/m of the next three stages in flight (their loads are plain global
+    // loads, so they need more lead than one stage to cover HBM latency)
+    uint32_t dm1[kLaneChunks], dm2[kLaneChunks], dm3[kLaneChunks];
+    load_dm(0, dm1);
+    load_dm(1, dm2);
+    load_dm(2, dm3);
+    float yacc[M];
+#pragma unroll
+    for (int t = 0; t < M; ++t) yacc[t] = 0.0f;
+
+    for (int it = 0; it < nstage; ++it) {
+        const int s = it % stages;
+        const int grp = it / nkc, kc = it - grp * nkc;
+        const int row = r0 + grp * kRowsPerStage + h;
+        uint32_t dm[kLaneChunks];
+#pragma unroll
+        for (int i = 0; i < kLaneChunks; ++i) {
+            dm[i] = dm1[i];
+            dm1[i] = dm2[i];
+            dm2[i] = dm3[i];
+        }
+        load_dm(it + 3, dm3);
+        if (!w4::mbar_wait(&full[s], (uint32_t)(it / stages) & 1u, abort_flag, err)) break;
+        if (row < r1) {
+            const uint8_t* src = smem + (size_t)s * kStageBytes + h * kChunkBytes;
+            const int nch = min(kChunkBytes, row_bytes - kc * kChunkBytes) >> 4;
+            const int c_base = kc * (kChunkBytes / 16);
+#pragma unroll
+            for (int i = 0; i < kLaneChunks; ++i) {
+                const int cl = j + 16 * i;
+                const bool live = cl < nch;  // predicated: chains of live chunks interleave
+                const int c = c_base + (live ? cl : 0);
+                const uint4 wq = live ? *reinterpret_cast<const uint4*>(src + cl * 16)
+                                      : make_uint4(0, 0, 0, 0);
+                int ah[M], al[M];
+#pragma unroll
+                for (int t = 0; t < M; ++t) {
+                    ah[t] = 0;
+                    al[t] = 0;
+                }
+#pragma unroll
+                for (int wi = 0; wi < 4; ++wi) {
+                    const uint32_t w = wi == 0 ? wq.x : wi == 1 ? wq.y : wi == 2 ? wq.z : wq.w;
+                    const uint32_t lo = w & 0x0F0F0F0Fu;         // codes of k = 0, 2, 4, 6
+                    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // codes of k = 1, 3, 5, 7
+#pragma unroll
+                    for (int t = 0; t < M; ++t) {
+                        // {Xh even k, Xh odd k, Xl even k, Xl odd k} of this word
+                        const uint4 xv = xq[((size_t)t * 4 + wi) * C + c];
+                        ah[t] = __dp4a((int)lo, (int)xv.x, ah[t]);
+                        ah[t] = __dp4a((int)hi, (int)xv.y, ah[t]);
+                        al[t] = (int)__dp4a(lo, xv.z, (unsigned)al[t]);
+                        al[t] = (int)__dp4a(hi, xv.w, (unsigned)al[t]);
+                    }
+                }
+                const float dd = __half2float(__ushort_as_half((unsigned short)(dm[i] & 0xFFFFu)));
+                const float mm = __half2float(__ushort_as_half((unsigned short)(dm[i] >> 16)));
+#pragma unroll
+                for (int t = 0; t < M; ++t) {
+                    const float qx = (float)(ah[t] * 256 + al[t]) * inv[t * C + c];
+                    const float v = fmaf(dd, qx, fmaf(mm, sx[t * C + c], yacc[t]));
+                    yacc[t] = live ? v : yacc[t];
+                }
+            }
+        }
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) w4::mbar_arrive(&empty[s]);
+        if (kc == nkc - 1) {
+            // row finished: reduce the 16 lanes (xor < 16 stays in the half-warp)
+#pragma unroll
+            for (int t = 0; t < M; ++t) {
+                float v = yacc[t];
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                if (row < r1 && j == t) {
+                    if (out_f32)
+                        reinterpret_cast<float*>(y)[(size_t)t * N + row] = v;
+                    else
+                        reinterpret_cast<__nv_bfloat16*>(y)[(size_t)t * N + row] =
+                            __float2bfloat16_rn(v);
+                }
+                yacc[t] = 0.0f;
+            }
+        }
+    }
+}
+
+// Stages of the code ring and resident CTAs per SM for M tokens: four stages
+// where the activation words leave room, and two CTAs per SM when both fit.
+struct Plan {
+    int stages, per_sm;
+    size_t smem;
+};
+
+Plan plan_for(int M, int C) {
+    Plan p{0, 0, 0};
+    for (int st = kMaxStages; st >= 2; --st) {
+        const size_t need = layout(M, C, st).total;
+        if (need <= (size_t)kSmemPerSm) {
+            p.stages = st;
+            p.smem = need;
+            // 228 KB of shared memory per SM, 1 KB of it reserved per CTA
+            p.per_sm = (M <= 4 && 2 * (need + 1024) <= (size_t)228 * 1024) ? 2 : 1;
+            return p;
+        }
+    }
+    return p;
+}
+
+template <int M>
+int launch_ring(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
+                const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
+    auto kern = w4_gemv_ring_kernel<M>;
+    const Plan pl = plan_for(M, K / 32);  // per_sm matches RingMinCtas<M>
+    if (pl.stages == 0) return W4_ERR_SHAPE;
+    static thread_local int attr_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return w4::cuda_fail(e);
+    if (attr_dev != dev) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemPerSm);
+        if (e != cudaSuccess) return w4::cuda_fail(e);
+        attr_dev = dev;
+    }
+    // contiguous, balanced row ranges: one per CTA
+    int grid = pl.per_sm * w4::sm_count();
+    if (grid > N) grid = N;
+    const int rows_per_cta = (N + grid - 1) / grid;
+    grid = (N + rows_per_cta - 1) / rows_per_cta;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kRingThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, codes, reinterpret_cast<const __half*>(d),
+                           reinterpret_cast<const __half*>(m), N, K, pl.stages, rows_per_cta, x,
+                           y, out_f32, w4::device_error_word());
+    if (e != cudaSuccess) return w4::cuda_fail(e);
+    return w4::launch_status();
+}
+
+
+template <int M>
+int dispatch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
+             const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
+    if ((size_t)N * (size_t)(K / 2) < kRingMaxCodeBytes && plan_for(M, K / 32).stages > 0)
+        return launch_ring<M>(codes, d, m, N, K, x, y, out_f32, st);
+    return dispatch_m<M>(codes, d, m, N, K, x, y, out_f32, st);
 }
 
 }  // namespace
@@ -470,13 +796,13 @@ extern "C" int w4_gemv(const uint8_t* codes, const uint16_t* d_f16, const uint16
     cudaStream_t st = (cudaStream_t)stream;
     const int n = (int)N, k = (int)K;
     switch (M) {
-        case 1: return dispatch_m<1>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 2: return dispatch_m<2>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 3: return dispatch_m<3>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 4: return dispatch_m<4>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 5: return dispatch_m<5>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 6: return dispatch_m<6>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 7: return dispatch_m<7>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        default: return dispatch_m<8>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        case 1: return dispatch<1>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        case 2: return dispatch<2>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        case 3: return dispatch<3>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        case 4: return dispatch<4>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        case 5: return dispatch<5>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        case 6: return dispatch<6>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        case 7: return dispatch<7>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
+        default: return dispatch<8>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
     }
 }
