@@ -534,14 +534,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // every epilogue thread reaches both barriers, aborted or not
                 const int tile = tmi * p.tiles_n + tni;
                 const int split = u % p.splits;
+                // partial tile layout: float4 [column quad][token row], so the 32
+                // lanes (consecutive rows) of a warp store 512 contiguous bytes
                 if (ok) {
-                    float* mine = p.partials +
-                                  (((size_t)tile * p.splits + split) * BM + row) * BN +
-                                  cs * kEpiCols;
+                    float4* mine = reinterpret_cast<float4*>(
+                                       p.partials + ((size_t)tile * p.splits + split) * BM * BN) +
+                                   (size_t)cs * (kEpiCols / 4) * BM + row;
 #pragma unroll
                     for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
-                        *reinterpret_cast<float4*>(mine + 4 * c4) = make_float4(
-                            yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
+                        mine[(size_t)c4 * BM] = make_float4(yv[4 * c4], yv[4 * c4 + 1],
+                                                            yv[4 * c4 + 2], yv[4 * c4 + 3]);
                 }
                 __threadfence();
                 asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -555,16 +557,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 store = store && last;
                 if (last) {
                     __threadfence();
-                    const float* base =
-                        p.partials + ((size_t)tile * p.splits * BM + row) * BN + cs * kEpiCols;
+                    const float4* base =
+                        reinterpret_cast<const float4*>(p.partials + (size_t)tile * p.splits * BM * BN) +
+                        (size_t)cs * (kEpiCols / 4) * BM + row;
 #pragma unroll
                     for (int c = 0; c < kEpiCols; ++c) yv[c] = 0.0f;
                     for (int q = 0; q < p.splits; ++q) {
-                        const float4* src =
-                            reinterpret_cast<const float4*>(base + (size_t)q * BM * BN);
+                        const float4* src = base + (size_t)q * (BM * BN / 4);
 #pragma unroll
                         for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
-                            const float4 v = __ldcg(src + c4);
+                            const float4 v = __ldcg(src + (size_t)c4 * BM);
                             yv[4 * c4] += v.x;
                             yv[4 * c4 + 1] += v.y;
                             yv[4 * c4 + 2] += v.z;
