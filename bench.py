@@ -59,6 +59,11 @@ def gemv_bytes(N: int, K: int, M: int, out_bytes: int = 2) -> int:
     return N * K // 2 + N * (K // GROUP) * 4 + M * K * 2 + M * N * out_bytes
 
 
+def w4a8_gemv_bytes(N: int, K: int, M: int, out_bytes: int = 2) -> int:
+    """Bytes the keep-quant GEMV must move: codes, d, m, qa, dx, S and y."""
+    return N * K // 2 + N * (K // GROUP) * 4 + M * K + M * (K // 32) * 8 + M * N * out_bytes
+
+
 def mmq_ops(M: int, N: int, K: int) -> int:
     return 2 * M * N * K
 
@@ -294,6 +299,40 @@ def time_gemv_sweep(torch, w4, wl, M, steps, warmup, stream):
     return elapsed, per, steps * len(SHAPES)
 
 
+def time_w4a8_gemv(torch, w4, wl, M, steps, stream):
+    """Keep-quant decode GEMV (int8 activation blocks from q8_quantize_act,
+    quantised once outside the timed launches): per-shape mean ms, each launch
+    its own CUDA graph between events, shapes in sweep order so the lm_head
+    between repeats of a shape keeps L2 from holding its weights."""
+    xs, ys = wl.xs(M)
+    acts = [w4.q8_quantize_act(x) for x in xs]
+    ncopy = len(wl.weights)
+
+    def run(c, s):
+        codes, d, m = wl.weights[c][s]
+        qa, dx, S = acts[s]
+        w4.w4a8_gemv(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=ys[s], stream=stream)
+
+    graphs = [[_capture(torch, stream, lambda c=c, s=s: run(c, s)) for s in range(len(SHAPES))]
+              for c in range(ncopy)]
+    with torch.cuda.stream(stream):
+        for c in range(ncopy):
+            for s in range(len(SHAPES)):
+                graphs[c][s].replay()
+        torch.cuda.synchronize()
+        evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in SHAPES]
+               for _ in range(steps)]
+        for i in range(steps):
+            for s in range(len(SHAPES)):
+                evs[i][s][0].record(stream)
+                graphs[i % ncopy][s].replay()
+                evs[i][s][1].record(stream)
+        torch.cuda.synchronize()
+    del graphs
+    return [statistics.mean(evs[i][s][0].elapsed_time(evs[i][s][1]) for i in range(steps))
+            for s in range(len(SHAPES))]
+
+
 def time_gemv_back_to_back(torch, w4, wl, s, reps, stream):
     """Steady-state duration of one shape's GEMV: `reps` launches in one CUDA
     graph, consecutive launches on alternating weight copies, event-timed on
@@ -522,6 +561,13 @@ def run_ours(args):
                                      "gbs": round(gemv_bytes(n, k, M) / (ms / 1e3) / 1e9, 1),
                                      "tok_per_s": round(M / (ms / 1e3), 1)}
                                     for (n, k), ms in zip(SHAPES, per)]
+        for M in (1, 4, 8):
+            per = time_w4a8_gemv(torch, w4, wl, M, max(3, args.steps // 2), stream)
+            extras[f"w4a8_gemv_m{M}"] = [
+                {"N": n, "K": k, "us": round(ms * 1e3, 2),
+                 "gbs": round(w4a8_gemv_bytes(n, k, M) / (ms / 1e3) / 1e9, 1),
+                 "tok_per_s": round(M / (ms / 1e3), 1)}
+                for (n, k), ms in zip(SHAPES, per)]
         del wl
         torch.cuda.empty_cache()
         mmq = time_mmq(torch, w4, dev, stream)

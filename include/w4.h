@@ -115,6 +115,24 @@ int w4_gemv(const uint8_t *codes, const uint16_t *d_f16,
             const uint16_t *x_bf16, int M, void *y, int out_dtype,
             void *stream);
 
+/* Decode GEMV on int8 activation blocks ("keep-quant" decode: the
+ * activations stay in the Q8_1-style blocks that q8_quantize_act produces, so
+ * the core of every 32-element block is an exact integer dot product, as in
+ * the decode arm of the GFX1100-TG200 campaign page that keeps the integer
+ * core bit-exact against the CPU).  It computes the W4A8 product of w4a8_mmq
+ * for decode batches:
+ *   P[t][n][b] = sum_{k in block b} q[n][k] * qa[t][k]      (exact int32)
+ *   y[t][n]    = sum_g ( d[n][g] * sum_{b in g} dx[t][b] * P[t][n][b]
+ *                        + m[n][g] * sum_{b in g} dx[t][b] * S[t][b] )
+ * scales applied in fp32.  codes/d/m: W[N][K] planes; qa int8 [M][K], dx fp32
+ * [M][K/32], bsum int32 [M][K/32]: the output of q8_quantize_act; y: [M][N]
+ * of out_dtype.  1 <= M <= 8, N >= 1, K >= 256, K % 256 == 0; every pointer
+ * 16-byte aligned.  Same validation and errors as w4_gemv. */
+int w4a8_gemv(const uint8_t *codes, const uint16_t *d_f16,
+              const uint16_t *m_f16, int64_t N, int64_t K, const int8_t *qa,
+              const float *dx, const int32_t *bsum, int M, void *y,
+              int out_dtype, void *stream);
+
 /* Quantise bf16 activations to int8 per block of 32 (the article's
  * "pre-quantise prefill activations to the Q8_1 MMQ layout"), with the
  * reading adopted for the unprinted rule:

@@ -28,7 +28,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for expected in ["w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "q8_quantize_act",
+    for expected in ["w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "w4a8_gemv",
+                     "q8_quantize_act",
                      "w4a8_mmq", "w4a8_mmq_workspace_size", "w4_status_string",
                      "w4_abi_version", "w4_last_cuda_error", "w4_check_device_error"]:
         assert expected in names
@@ -71,6 +72,18 @@ def test_gemv_validation(lib):
     assert f(FAKE, FAKE, FAKE, 256, 512, None, 1, FAKE, 0, None) == L.W4_ERR_NULL
     assert f(MIS, FAKE, FAKE, 256, 512, FAKE, 1, FAKE, 0, None) == L.W4_ERR_ALIGN
     assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, 1, MIS, 0, None) == L.W4_ERR_ALIGN
+
+
+def test_w4a8_gemv_validation(lib):
+    from w4_quant_matmul_b200 import _lib as L
+    f = lib.w4a8_gemv
+    assert f(FAKE, FAKE, FAKE, 256, 300, FAKE, FAKE, FAKE, 1, FAKE, 0, None) == L.W4_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, FAKE, FAKE, 9, FAKE, 0, None) == L.W4_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, FAKE, FAKE, 1, FAKE, 7, None) == L.W4_ERR_SHAPE
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, None, FAKE, 1, FAKE, 0, None) == L.W4_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, FAKE, None, 1, FAKE, 0, None) == L.W4_ERR_NULL
+    assert f(FAKE, FAKE, FAKE, 256, 512, MIS, FAKE, FAKE, 1, FAKE, 0, None) == L.W4_ERR_ALIGN
+    assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, MIS, FAKE, 1, FAKE, 0, None) == L.W4_ERR_ALIGN
 
 
 def test_pack_and_quantizer_validation(lib):

@@ -11,6 +11,7 @@ Entry points (same names as the C ABI):
     w4_pack_codes(q)                        -> codes
     w4_unpack(codes, K)                     -> q
     w4_gemv(codes, d, m, x, out_dtype)      -> y
+    w4a8_gemv(codes, d, m, qa, dx, bsum, out_dtype) -> y   (int8 activations, M <= 8)
     q8_quantize_act(x)                      -> qa, dx, bsum
     w4a8_mmq(codes, d, m, qa, dx, bsum, out_dtype) -> y
     w4a8_mmq_static(codes, d, m, qa, dx, bsum, out_dtype) -> y   (no workspace)
@@ -22,7 +23,7 @@ from __future__ import annotations
 from ._lib import (LibraryMissing, W4_OK, W4_OUT_BF16, W4_OUT_F32, load, status_string)
 
 __all__ = [
-    "W4Error", "LibraryMissing", "w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv",
+    "W4Error", "LibraryMissing", "w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "w4a8_gemv",
     "q8_quantize_act", "w4a8_mmq", "w4a8_mmq_static", "w4a8_mmq_workspace_size",
     "w4_check_device_error",
     "w4_abi_version", "lib",
@@ -163,6 +164,28 @@ def w4_gemv(codes, d, m, x, out_dtype=None, y=None, stream=None):
                         device=x.device)
     _check(load().w4_gemv(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x), M, _ptr(y), oc,
                           _stream(stream)), "w4_gemv")
+    return y
+
+
+def w4a8_gemv(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, stream=None):
+    """y[M,N] for 1 <= M <= 8 from W4-G256 weights and int8 activation blocks
+    (the output of q8_quantize_act): exact int32 block dot products, scales in fp32."""
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    _need(codes, torch.uint8, "codes")
+    _need(d, torch.float16, "d")
+    _need(m, torch.float16, "m")
+    _need(qa, torch.int8, "qa")
+    _need(dx, torch.float32, "dx")
+    _need(bsum, torch.int32, "bsum")
+    N = codes.shape[0]
+    M, K = qa.shape
+    oc = _out_code(out_dtype)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32 if oc == W4_OUT_F32 else torch.bfloat16,
+                        device=qa.device)
+    _check(load().w4a8_gemv(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(qa), _ptr(dx), _ptr(bsum),
+                            M, _ptr(y), oc, _stream(stream)), "w4a8_gemv")
     return y
 
 

@@ -119,7 +119,7 @@ __device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __res
     }
 }
 
-template <int M, int RH, int U>
+template <int M, int RH, int U, bool A8>
 __device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4* __restrict__ xq,
                                               const float* __restrict__ sx,
                                               const float* __restrict__ inv, int C, int c0,
@@ -153,8 +153,10 @@ __device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4
                 for (int t = 0; t < M; ++t) {
                     ah[t][i] = __dp4a((int)lo, (int)xv[t].x, ah[t][i]);
                     ah[t][i] = __dp4a((int)hi, (int)xv[t].y, ah[t][i]);
-                    al[t][i] = (int)__dp4a(lo, xv[t].z, (unsigned)al[t][i]);
-                    al[t][i] = (int)__dp4a(hi, xv[t].w, (unsigned)al[t][i]);
+                    if constexpr (!A8) {
+                        al[t][i] = (int)__dp4a(lo, xv[t].z, (unsigned)al[t][i]);
+                        al[t][i] = (int)__dp4a(hi, xv[t].w, (unsigned)al[t][i]);
+                    }
                 }
             }
         }
@@ -165,7 +167,8 @@ __device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4
             for (int i = 0; i < RH; ++i) {
                 const float dd = __half2float(__ushort_as_half((unsigned short)(b.dm[u][i] & 0xFFFFu)));
                 const float mm = __half2float(__ushort_as_half((unsigned short)(b.dm[u][i] >> 16)));
-                const float qx = (float)(ah[t][i] * 256 + al[t][i]) * iv;
+                // A8: the exact block dot P times dx; else (sum q X) / sigma
+                const float qx = (A8 ? (float)ah[t][i] : (float)(ah[t][i] * 256 + al[t][i])) * iv;
                 yacc[t][i] = fmaf(dd, qx, fmaf(mm, s, yacc[t][i]));
             }
         }
@@ -225,6 +228,35 @@ __device__ __forceinline__ void stage_quarter(uint4 raw, bool live, uint4* __res
     }
 }
 
+// Activations: bf16 x [M][K] (A8 = false), or int8 blocks of 32 with their
+// scales and sums (A8 = true: qa [M][K], dx and S [M][K/32]).
+struct Act {
+    const void* x;
+    const float* dx;
+    const int32_t* S;
+};
+
+// One int8 activation block (32 values of token t, chunk c) -> the words the
+// dp4a loop reads: word wi holds the bytes of k = 8 wi + {0, 2, 4, 6} (.x) and
+// k = 8 wi + {1, 3, 5, 7} (.y), matching the low / high nibbles of a code word;
+// the chunk's "sum" slot holds dx * S and its "inverse scale" slot dx.
+__device__ __forceinline__ void stage_block_a8(const Act& a, int C, int t, int c,
+                                               uint4* __restrict__ xq, float* __restrict__ sx,
+                                               float* __restrict__ inv) {
+    const uint4* src = reinterpret_cast<const uint4*>(
+        reinterpret_cast<const int8_t*>(a.x) + ((size_t)t * C + c) * 32);
+    const uint4 q0 = __ldg(src), q1 = __ldg(src + 1);
+    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi)
+        xq[((size_t)t * 4 + wi) * C + c] =
+            make_uint4(__byte_perm(w[2 * wi], w[2 * wi + 1], 0x6420),
+                       __byte_perm(w[2 * wi], w[2 * wi + 1], 0x7531), 0u, 0u);
+    const float dxv = __ldg(a.dx + (size_t)t * C + c);
+    sx[t * C + c] = dxv * (float)__ldg(a.S + (size_t)t * C + c);
+    inv[t * C + c] = dxv;
+}
+
 // Resident CTAs per SM the register allocation is sized for: small M needs
 // many warps in flight to cover HBM latency; large M needs the registers.
 template <int M>
@@ -232,10 +264,10 @@ struct MinCtas {
     static constexpr int value = M == 1 ? 3 : (M <= 4 ? 2 : 1);
 };
 
-template <int M, int RH, int U>
+template <int M, int RH, int U, bool A8>
 __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
-    int N, int K, int KS, const uint16_t* __restrict__ x, void* __restrict__ y, int out_f32) {
+    int N, int K, int KS, const Act act, void* __restrict__ y, int out_f32) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int C = K >> 5;  // 32-code chunks per row
     const int G = K >> 8;  // groups per row
@@ -276,17 +308,23 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
     pdl_wait();
 
     // ---- activation words, chunk sums and scales, once per CTA ----
-    const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
-    for (int base = 0; base < nq; base += kThreads) {
-        const int v = base + threadIdx.x;
-        const bool live = v < nq;
-        const int vv = live ? v : 0;
-        const int t = vv / (C * 4);
-        const int r = vv - t * C * 4;
-        const int c = r >> 2, q4 = r & 3;
-        const uint4 raw = live ? __ldg(reinterpret_cast<const uint4*>(x) + vv) : make_uint4(0, 0, 0, 0);
-        stage_quarter(raw, live, &xq[((size_t)t * 4 + q4) * C + c], &sx[t * C + c],
-                      &inv[t * C + c], q4);
+    if constexpr (A8) {
+        for (int v = threadIdx.x; v < M * C; v += kThreads)
+            stage_block_a8(act, C, v / C, v - (v / C) * C, xq, sx, inv);
+    } else {
+        const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
+        for (int base = 0; base < nq; base += kThreads) {
+            const int v = base + threadIdx.x;
+            const bool live = v < nq;
+            const int vv = live ? v : 0;
+            const int t = vv / (C * 4);
+            const int r = vv - t * C * 4;
+            const int c = r >> 2, q4 = r & 3;
+            const uint4 raw = live ? __ldg(reinterpret_cast<const uint4*>(act.x) + vv)
+                                   : make_uint4(0, 0, 0, 0);
+            stage_quarter(raw, live, &xq[((size_t)t * 4 + q4) * C + c], &sx[t * C + c],
+                          &inv[t * C + c], q4);
+        }
     }
     __syncthreads();
     pdl_launch_dependents();
@@ -302,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
         if (active) {
             for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
                 if (c0 != cs + j) load_batch(bt, codes, d, m, rows, row_bytes, G, c0, ce);
-                consume_batch<M, RH, U>(bt, xq, sx, inv, C, c0, ce, yacc);
+                consume_batch<M, RH, U, A8>(bt, xq, sx, inv, C, c0, ce, yacc);
             }
         }
         // reduce the 16 lanes of the half-warp (xor < 16 stays inside it)
@@ -379,11 +417,11 @@ size_t smem_bytes(int M, int C, int KS, int RH) {
            (KS > 1 ? (size_t)KS * rows_per_cta * M * 4 : 0);
 }
 
-template <int M, int RH>
+template <int M, int RH, bool A8>
 int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K, int KS,
-           const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
+           const Act& x, void* y, int out_f32, cudaStream_t st) {
     constexpr int U = 8 / RH;
-    auto kern = w4_gemv_rows_kernel<M, RH, U>;
+    auto kern = w4_gemv_rows_kernel<M, RH, U, A8>;
     const int C = K / 32;
     const size_t smem = smem_bytes(M, C, KS, RH);
     // Per-instantiation cache: one device, a few shared-memory sizes.
@@ -448,18 +486,18 @@ void pick_split(int N, int C, int sms, int* rh, int* ks) {
     *ks = k;
 }
 
-template <int M>
+template <int M, bool A8>
 int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
-               const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
+               const Act& x, void* y, int out_f32, cudaStream_t st) {
     int rh, ks;
     pick_split(N, K / 32, w4::sm_count(), &rh, &ks);
     if (M >= 4 && rh > 2) rh = 2;  // register budget: M * RH accumulators twice
     if (smem_bytes(M, K / 32, ks, rh) > (size_t)kSmemBudget) ks = 1;
     if constexpr (M < 4) {
-        if (rh == 4) return launch_rows<M, 4>(codes, d, m, N, K, ks, x, y, out_f32, st);
+        if (rh == 4) return launch_rows<M, 4, A8>(codes, d, m, N, K, ks, x, y, out_f32, st);
     }
-    if (rh >= 2) return launch_rows<M, 2>(codes, d, m, N, K, ks, x, y, out_f32, st);
-    return launch_rows<M, 1>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    if (rh >= 2) return launch_rows<M, 2, A8>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    return launch_rows<M, 1, A8>(codes, d, m, N, K, ks, x, y, out_f32, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -499,11 +537,11 @@ struct RingMinCtas {
     static constexpr int value = M <= 4 ? 2 : 1;
 };
 
-template <int M>
+template <int M, bool A8>
 __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_ring_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
-    int N, int K, int stages, int rows_per_cta, const uint16_t* __restrict__ x,
-    void* __restrict__ y, int out_f32, int* err) {
+    int N, int K, int stages, int rows_per_cta, const Act act, void* __restrict__ y, int out_f32,
+    int* err) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int C = K >> 5;          // 32-code chunks per row
     const int G = K >> 8;          // groups per row
@@ -573,26 +611,32 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
 
     // activation words, chunk sums and scales, once per CTA; each thread issues
     // up to four 16-byte loads before converting any
-    const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
     constexpr int kCons = 32 * kRingWarps;
-    for (int base = 0; base < nq; base += 4 * kCons) {
-        uint4 raw[4];
+    if constexpr (A8) {
+        for (int v = threadIdx.x; v < M * C; v += kCons)
+            stage_block_a8(act, C, v / C, v - (v / C) * C, xq, sx, inv);
+    } else {
+        const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
+        for (int base = 0; base < nq; base += 4 * kCons) {
+            uint4 raw[4];
 #pragma unroll
-        for (int p4 = 0; p4 < 4; ++p4) {
-            const int v = base + p4 * kCons + threadIdx.x;
-            raw[p4] = v < nq ? __ldg(reinterpret_cast<const uint4*>(x) + v) : make_uint4(0, 0, 0, 0);
-        }
+            for (int p4 = 0; p4 < 4; ++p4) {
+                const int v = base + p4 * kCons + threadIdx.x;
+                raw[p4] = v < nq ? __ldg(reinterpret_cast<const uint4*>(act.x) + v)
+                                 : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-        for (int p4 = 0; p4 < 4; ++p4) {
-            if (base + p4 * kCons >= nq) break;  // uniform across the consumers
-            const int v = base + p4 * kCons + threadIdx.x;
-            const bool live = v < nq;
-            const int vv = live ? v : 0;
-            const int t = vv / (C * 4);
-            const int r = vv - t * C * 4;
-            const int c = r >> 2, q4 = r & 3;
-            stage_quarter(raw[p4], live, &xq[((size_t)t * 4 + q4) * C + c], &sx[t * C + c],
-                          &inv[t * C + c], q4);
+            for (int p4 = 0; p4 < 4; ++p4) {
+                if (base + p4 * kCons >= nq) break;  // uniform across the consumers
+                const int v = base + p4 * kCons + threadIdx.x;
+                const bool live = v < nq;
+                const int vv = live ? v : 0;
+                const int t = vv / (C * 4);
+                const int r = vv - t * C * 4;
+                const int c = r >> 2, q4 = r & 3;
+                stage_quarter(raw[p4], live, &xq[((size_t)t * 4 + q4) * C + c], &sx[t * C + c],
+                              &inv[t * C + c], q4);
+            }
         }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
@@ -669,15 +713,18 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
                         const uint4 xv = xq[((size_t)t * 4 + wi) * C + c];
                         ah[t] = __dp4a((int)lo, (int)xv.x, ah[t]);
                         ah[t] = __dp4a((int)hi, (int)xv.y, ah[t]);
-                        al[t] = (int)__dp4a(lo, xv.z, (unsigned)al[t]);
-                        al[t] = (int)__dp4a(hi, xv.w, (unsigned)al[t]);
+                        if constexpr (!A8) {
+                            al[t] = (int)__dp4a(lo, xv.z, (unsigned)al[t]);
+                            al[t] = (int)__dp4a(hi, xv.w, (unsigned)al[t]);
+                        }
                     }
                 }
                 const float dd = __half2float(__ushort_as_half((unsigned short)(dm[i] & 0xFFFFu)));
                 const float mm = __half2float(__ushort_as_half((unsigned short)(dm[i] >> 16)));
 #pragma unroll
                 for (int t = 0; t < M; ++t) {
-                    const float qx = (float)(ah[t] * 256 + al[t]) * inv[t * C + c];
+                    const float qx =
+                        (A8 ? (float)ah[t] : (float)(ah[t] * 256 + al[t])) * inv[t * C + c];
                     const float v = fmaf(dd, qx, fmaf(mm, sx[t * C + c], yacc[t]));
                     yacc[t] = live ? v : yacc[t];
                 }
@@ -729,10 +776,10 @@ Plan plan_for(int M, int C) {
     return p;
 }
 
-template <int M>
+template <int M, bool A8>
 int launch_ring(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
-                const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
-    auto kern = w4_gemv_ring_kernel<M>;
+                const Act& x, void* y, int out_f32, cudaStream_t st) {
+    auto kern = w4_gemv_ring_kernel<M, A8>;
     const Plan pl = plan_for(M, K / 32);  // per_sm matches RingMinCtas<M>
     if (pl.stages == 0) return W4_ERR_SHAPE;
     static thread_local int attr_dev = -1;
@@ -768,12 +815,43 @@ int launch_ring(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int 
 }
 
 
-template <int M>
+template <int M, bool A8>
 int dispatch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
-             const uint16_t* x, void* y, int out_f32, cudaStream_t st) {
+             const Act& x, void* y, int out_f32, cudaStream_t st) {
     if ((size_t)N * (size_t)(K / 2) < kRingMaxCodeBytes && plan_for(M, K / 32).stages > 0)
-        return launch_ring<M>(codes, d, m, N, K, x, y, out_f32, st);
-    return dispatch_m<M>(codes, d, m, N, K, x, y, out_f32, st);
+        return launch_ring<M, A8>(codes, d, m, N, K, x, y, out_f32, st);
+    return dispatch_m<M, A8>(codes, d, m, N, K, x, y, out_f32, st);
+}
+
+template <bool A8>
+int dispatch_any_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
+                   const Act& x, int M, void* y, int out_f32, cudaStream_t st) {
+    switch (M) {
+        case 1: return dispatch<1, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        case 2: return dispatch<2, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        case 3: return dispatch<3, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        case 4: return dispatch<4, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        case 5: return dispatch<5, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        case 6: return dispatch<6, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        case 7: return dispatch<7, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        default: return dispatch<8, A8>(codes, d, m, N, K, x, y, out_f32, st);
+    }
+}
+
+// Host validation shared by both entry points; W4_OK if the call may launch.
+int validate(const void* codes, const void* d, const void* m, int64_t N, int64_t K,
+             const void* a0, const void* a1, const void* a2, int M, const void* y,
+             int out_dtype) {
+    if (M < 1 || M > 8 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
+    if (N > (int64_t)1 << 30 || K > (int64_t)1 << 20) return W4_ERR_SHAPE;
+    if (out_dtype != W4_OUT_BF16 && out_dtype != W4_OUT_F32) return W4_ERR_SHAPE;
+    if (!codes || !d || !m || !a0 || !a1 || !a2 || !y) return W4_ERR_NULL;
+    if (!w4::aligned16(codes) || !w4::aligned16(d) || !w4::aligned16(m) ||
+        !w4::aligned16(a0) || !w4::aligned16(a1) || !w4::aligned16(a2) || !w4::aligned16(y))
+        return W4_ERR_ALIGN;
+    // the activation words must fit the shared-memory stage
+    if (smem_bytes(M, (int)(K / 32), 1, 1) > (size_t)kSmemBudget) return W4_ERR_SHAPE;
+    return w4::check_device();
 }
 
 }  // namespace
@@ -781,28 +859,19 @@ int dispatch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, 
 extern "C" int w4_gemv(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
                        int64_t N, int64_t K, const uint16_t* x_bf16, int M, void* y,
                        int out_dtype, void* stream) {
-    if (M < 1 || M > 8 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
-    if (N > (int64_t)1 << 30 || K > (int64_t)1 << 20) return W4_ERR_SHAPE;
-    if (out_dtype != W4_OUT_BF16 && out_dtype != W4_OUT_F32) return W4_ERR_SHAPE;
-    if (!codes || !d_f16 || !m_f16 || !x_bf16 || !y) return W4_ERR_NULL;
-    if (!w4::aligned16(codes) || !w4::aligned16(d_f16) || !w4::aligned16(m_f16) ||
-        !w4::aligned16(x_bf16) || !w4::aligned16(y))
-        return W4_ERR_ALIGN;
-    // x (M*K bf16) and its chunk sums must fit the shared-memory stage
-    if (smem_bytes(M, (int)(K / 32), 1, 1) > (size_t)kSmemBudget) return W4_ERR_SHAPE;
-    int rc = w4::check_device();
+    const int rc = validate(codes, d_f16, m_f16, N, K, x_bf16, x_bf16, x_bf16, M, y, out_dtype);
     if (rc != W4_OK) return rc;
-    const int out_f32 = out_dtype == W4_OUT_F32;
-    cudaStream_t st = (cudaStream_t)stream;
-    const int n = (int)N, k = (int)K;
-    switch (M) {
-        case 1: return dispatch<1>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 2: return dispatch<2>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 3: return dispatch<3>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 4: return dispatch<4>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 5: return dispatch<5>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 6: return dispatch<6>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        case 7: return dispatch<7>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-        default: return dispatch<8>(codes, d_f16, m_f16, n, k, x_bf16, y, out_f32, st);
-    }
+    const Act act{x_bf16, nullptr, nullptr};
+    return dispatch_any_m<false>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
+                                 out_dtype == W4_OUT_F32, (cudaStream_t)stream);
+}
+
+extern "C" int w4a8_gemv(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
+                         int64_t N, int64_t K, const int8_t* qa, const float* dx,
+                         const int32_t* bsum, int M, void* y, int out_dtype, void* stream) {
+    const int rc = validate(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype);
+    if (rc != W4_OK) return rc;
+    const Act act{qa, dx, bsum};
+    return dispatch_any_m<true>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
+                                out_dtype == W4_OUT_F32, (cudaStream_t)stream);
 }
