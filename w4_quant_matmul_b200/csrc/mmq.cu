@@ -98,10 +98,18 @@ struct Smem {
     static constexpr int bp = b + STAGES * B_BYTES;
     static constexpr int bias = bp + STAGES * BP_BYTES;  // bias MMA operands (A, B)
     static constexpr int bars = bias + 2 * BIAS_BYTES;   // uint64 barriers
-    static constexpr int nbars = 3 * STAGES + 2 * NPAIR + 1;
+    static constexpr int nbars = 3 * STAGES + 2 * NPAIR + 1 + 4;
     static constexpr int misc = bars + nbars * 8;        // tmem base, abort flag
     static constexpr int dm = (misc + 16 + 15) & ~15;    // fp32 d[G][BN], m[G][BN]
-    static size_t total(int G) { return (size_t)dm + (size_t)2 * G * BN * 4 + 1024; }
+    // ring of per-group activation scales and block sums (two slots of
+    // dx fp32 [128 tokens][8] + S int32 [128][8]), after d and m
+    static constexpr int kScSlotBytes = 2 * BM * 8 * 4;
+    __host__ __device__ static size_t sc(int G) {
+        return ((size_t)dm + (size_t)2 * G * BN * 4 + 127) & ~(size_t)127;
+    }
+    static size_t total(int G, bool ring) {
+        return sc(G) + (ring ? 2 * (size_t)kScSlotBytes : 0) + 1024;
+    }
 };
 
 struct Params {
@@ -114,6 +122,7 @@ struct Params {
     int out_f32;
     int* err;
     int splits;            // K slices per output tile (1 = no split)
+    int sc_ring;           // 1: per-group dx/S arrive by TMA in a shared ring
     int tiles_n;           // output tiles along N
     int units;             // tiles * splits work units (CTAs loop over them)
     int* counters;         // [tiles] arrival counters (split > 1), zeroed before launch
@@ -188,7 +197,9 @@ __device__ __forceinline__ void tmem_wait_ld() {
 
 __global__ void __launch_bounds__(kThreads, 1)
     w4a8_mmq_kernel(const __grid_constant__ CUtensorMap tm_a,
-                    const __grid_constant__ CUtensorMap tm_b, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_dx,
+                    const __grid_constant__ CUtensorMap tm_s, const Params p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment of the operand tiles (128B swizzle atoms).
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -203,12 +214,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tfull = bars + 3 * STAGES;     // TMEM buffer pair written
     uint64_t* tempty = tfull + NPAIR;        // TMEM buffer pair read out
     uint64_t* drain = tempty + NPAIR;        // final MMA completion
+    uint64_t* scfull = drain + 1;            // a group's dx/S landed in its slot
+    uint64_t* scempty = scfull + 2;          // the epilogue has read the slot
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Smem::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
     volatile int* last_flag = abort_flag + 1;
     float* d_s = reinterpret_cast<float*>(smem + Smem::dm);
     const int G = p.K / 256;
     float* m_s = d_s + G * BN;
+    uint8_t* sc = smem + Smem::sc(G);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -236,6 +250,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             w4::mbar_init(&tempty[i], kEpiWarps);
         }
         w4::mbar_init(drain, 1);
+        for (int i = 0; i < 2; ++i) {
+            w4::mbar_init(&scfull[i], 1);
+            w4::mbar_init(&scempty[i], kEpiWarps);
+        }
         *abort_flag = 0;
         w4::fence_mbar_init();
     }
@@ -266,12 +284,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (w4::elect_one()) {
                 w4::prefetch_tmap(&tm_a);
                 w4::prefetch_tmap(&tm_b);
+                if (p.sc_ring) {
+                    w4::prefetch_tmap(&tm_dx);
+                    w4::prefetch_tmap(&tm_s);
+                }
                 int it = 0;  // global stage counter
+                int gi = 0;  // groups whose scales were issued
                 bool ok = true;
                 for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                     int tmi, tni, gb, ge;
                     unit_of(u, tmi, tni, gb, ge);
                     for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
+                        if (p.sc_ring && (kg & 1) == 0) {
+                            // the group's dx and S for the tile's 128 tokens, ahead of
+                            // its first stage (rows past M are zero-filled)
+                            const int slot = gi & 1;
+                            if (!w4::mbar_wait(&scempty[slot], ((uint32_t)(gi >> 1) & 1u) ^ 1u,
+                                               abort_flag, p.err)) {
+                                ok = false;
+                                break;
+                            }
+                            uint8_t* dst = sc + slot * Smem::kScSlotBytes;
+                            w4::mbar_arrive_expect_tx(&scfull[slot], Smem::kScSlotBytes);
+                            w4::tma_load_2d(dst, &tm_dx, &scfull[slot], (kg >> 1) * 8, tmi * BM);
+                            w4::tma_load_2d(dst + Smem::kScSlotBytes / 2, &tm_s, &scfull[slot],
+                                            (kg >> 1) * 8, tmi * BM);
+                            ++gi;
+                        }
                         const int s = it % STAGES;
                         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
                         if (!w4::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err)) {
@@ -287,6 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // drain: every issued load must land before the CTA exits
                 for (int k = it - STAGES < 0 ? 0 : it - STAGES; k < it; ++k)
                     w4::mbar_wait(&full[k % STAGES], (uint32_t)(k / STAGES) & 1u, nullptr, p.err);
+                for (int k = gi - 2 < 0 ? 0 : gi - 2; k < gi; ++k)
+                    w4::mbar_wait(&scfull[k & 1], (uint32_t)(k >> 1) & 1u, nullptr, p.err);
             }
         } else if (warp == 1) {
             // ---------------- MMA issuer ----------------
@@ -396,6 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cs * kEpiCols);
 
         int it = 0;
+        int gi = 0;  // groups started (the scale ring's slot sequence)
         bool ok = true;
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             int tmi, tni, g_begin, g_end;
@@ -444,11 +486,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i) dxg[i] = 0.0f;
                     tmin = 0.0f;
-                    if (t_live) {
+                    float4 sa4[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+                    int4 ss4[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};
+                    if (p.sc_ring) {
+                        // this token's 8 scales and sums, brought in by TMA
+                        const int slot = gi & 1;
+                        if (!w4::mbar_wait(&scfull[slot], (uint32_t)(gi >> 1) & 1u, abort_flag,
+                                           p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint8_t* src = sc + slot * Smem::kScSlotBytes;
+                        sa4[0] = reinterpret_cast<const float4*>(src)[2 * row];
+                        sa4[1] = reinterpret_cast<const float4*>(src)[2 * row + 1];
+                        ss4[0] = reinterpret_cast<const int4*>(src + Smem::kScSlotBytes / 2)[2 * row];
+                        ss4[1] =
+                            reinterpret_cast<const int4*>(src + Smem::kScSlotBytes / 2)[2 * row + 1];
+                        __syncwarp();
+                        if (lane == 0) w4::mbar_arrive(&scempty[slot]);
+                    } else if (t_live) {
 #pragma unroll
                         for (int h4 = 0; h4 < 2; ++h4) {
-                            const float4 a = __ldg(reinterpret_cast<const float4*>(dx_row + g * 8) + h4);
-                            const int4 sv = __ldg(reinterpret_cast<const int4*>(s_row + g * 8) + h4);
+                            sa4[h4] = __ldg(reinterpret_cast<const float4*>(dx_row + g * 8) + h4);
+                            ss4[h4] = __ldg(reinterpret_cast<const int4*>(s_row + g * 8) + h4);
+                        }
+                    }
+                    ++gi;
+                    {
+#pragma unroll
+                        for (int h4 = 0; h4 < 2; ++h4) {
+                            const float4 a = sa4[h4];
+                            const int4 sv = ss4[h4];
                             dxg[4 * h4] = a.x;
                             dxg[4 * h4 + 1] = a.y;
                             dxg[4 * h4 + 2] = a.z;
@@ -662,6 +730,24 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D tensor map over a dense row-major [rows][cols] matrix of 4-byte elements
+// (fp32 dx or int32 S), no swizzle; rows past the end read as zero.
+bool make_map_4b(CUtensorMap* map, const void* base, CUtensorMapDataType type, uint64_t cols,
+                 uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 4};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Usable dynamic shared memory per CTA on sm_100.
+constexpr size_t kSmemMax = 227 * 1024;
+
 // K slices per output tile.  Cost model in units of one 256-group of MMA work
 // per CTA: waves(tiles * S over the SMs) * (groups per slice + fixed cost of a
 // CTA's fill, drain and epilogue), each slice keeping >= 4 groups.
@@ -734,14 +820,28 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
         return W4_ERR_CUDA;
 
     const int G = (int)(K / 256);
-    const size_t smem = Smem::total(G);
+    // the scale ring when it fits next to d and m (every K up to 42 groups)
+    const bool ring = Smem::total(G, true) <= kSmemMax;
+    const size_t smem = Smem::total(G, ring);
+    CUtensorMap mdx, ms;
+    if (ring) {
+        // dx and S are [M][K/32]: row stride K/8 bytes (a multiple of 16), box 8 x 128
+        if (!make_map_4b(&mdx, dx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)K / 32,
+                         (uint64_t)M, 8, BM) ||
+            !make_map_4b(&ms, bsum, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)K / 32, (uint64_t)M,
+                         8, BM))
+            return W4_ERR_CUDA;
+    } else {
+        mdx = ma;  // unused by the kernel
+        ms = ma;
+    }
     static thread_local int attr_dev = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return w4::cuda_fail(e);
     if (attr_dev != dev) {
         e = cudaFuncSetAttribute(w4a8_mmq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Smem::total(kMaxGroups));
+                                 (int)kSmemMax);
         if (e != cudaSuccess) return w4::cuda_fail(e);
         attr_dev = dev;
     }
@@ -757,6 +857,7 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     prm.out_f32 = out_dtype == W4_OUT_F32;
     prm.err = err;
     prm.splits = splits;
+    prm.sc_ring = ring ? 1 : 0;
     prm.counters = nullptr;
     prm.partials = nullptr;
     if (splits > 1) {
@@ -769,7 +870,7 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     prm.tiles_n = (int)((N + BN - 1) / BN);
     prm.units = (int)(tiles * splits);
     const int grid = prm.units < w4::sm_count() ? prm.units : w4::sm_count();
-    w4a8_mmq_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, prm);
+    w4a8_mmq_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, mdx, ms, prm);
     return w4::launch_status();
 }
 
