@@ -112,7 +112,7 @@ def test_mmq_validation(lib):
         return f(*a)
 
     assert call(a4=384) == L.W4_ERR_SHAPE          # K % 256
-    assert call(a4=256 * 57) == L.W4_ERR_SHAPE     # K above the supported maximum
+    assert call(a4=256 * 513) == L.W4_ERR_SHAPE    # K above the supported maximum
     assert call(a8=0) == L.W4_ERR_SHAPE            # M
     assert call(a10=3) == L.W4_ERR_SHAPE           # out dtype
     assert call(a5=None) == L.W4_ERR_NULL

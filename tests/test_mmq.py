@@ -92,6 +92,15 @@ def test_extreme_integer_products(torch, w4, orc, scales):
     _both(torch, w4, orc, codes, d, m, qa, dx, S, what="extreme")
 
 
+def test_long_k(torch, w4, orc):
+    # K = 16384 (64 groups): past the per-tile d/m staging limit of earlier
+    # versions; every output against the oracle, split-K or not
+    M, N, K = 130, 200, 16384
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=21)
+    qa, dx, S = orc.q8_quantize(synth.outlier_activations(M, K, seed=22))
+    _both(torch, w4, orc, codes, d, m, qa, dx, S, what="K16384")
+
+
 def test_zero_blocks_and_zero_scales(torch, w4, orc):
     M, N, K = 140, 130, 512
     codes, d, m = synth.quantized_weights_direct(N, K, seed=2)

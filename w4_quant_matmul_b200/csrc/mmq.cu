@@ -54,8 +54,8 @@
 // Requires |dx| < 2^100 (activations far beyond any fp16/bf16 model range
 // would overflow the scaled products).
 //
-// Registers are rebalanced with setmaxnreg: 40 per thread for warps 0-3, 232
-// for the epilogue (128*40 + 256*232 = 384*168, the launch allotment).
+// Registers are rebalanced with setmaxnreg: 48 per thread for warps 0-3, 224
+// for the epilogue (128*48 + 256*224 <= 384*168, the launch allotment).
 // K slices (split-K) write fp32 partial tiles to the caller's workspace; the
 // CTA that finishes a tile last sums the partials in slice order (bitwise
 // deterministic) and stores y.
@@ -88,7 +88,7 @@ constexpr int A_BYTES = BM * BK;
 constexpr int B_BYTES = BN * BK;
 constexpr int BP_BYTES = BN * BK / 2;
 constexpr int TMEM_COLS = NTB * BN;   // 512
-constexpr int kMaxGroups = 56;        // K <= 14336 (shared memory for d, m)
+constexpr int kMaxGroups = 512;       // K <= 131072 (shared memory does not depend on K)
 
 static_assert(TMEM_COLS == 512, "TMEM allocation must be a power of two <= 512");
 
@@ -98,18 +98,14 @@ struct Smem {
     static constexpr int bp = b + STAGES * B_BYTES;
     static constexpr int bias = bp + STAGES * BP_BYTES;  // bias MMA operands (A, B)
     static constexpr int bars = bias + 2 * BIAS_BYTES;   // uint64 barriers
-    static constexpr int nbars = 3 * STAGES + 2 * NPAIR + 1 + 4;
+    static constexpr int nbars = 3 * STAGES + 2 * NPAIR + 1 + 4 + 4;
     static constexpr int misc = bars + nbars * 8;        // tmem base, abort flag
-    static constexpr int dm = (misc + 16 + 15) & ~15;    // fp32 d[G][BN], m[G][BN]
+    static constexpr int dm = (misc + 16 + 15) & ~15;    // fp32 [2 slots][d, m][BN]
     // ring of per-group activation scales and block sums (two slots of
     // dx fp32 [128 tokens][8] + S int32 [128][8]), after d and m
     static constexpr int kScSlotBytes = 2 * BM * 8 * 4;
-    __host__ __device__ static size_t sc(int G) {
-        return ((size_t)dm + (size_t)2 * G * BN * 4 + 127) & ~(size_t)127;
-    }
-    static size_t total(int G, bool ring) {
-        return sc(G) + (ring ? 2 * (size_t)kScSlotBytes : 0) + 1024;
-    }
+    static constexpr int sc = (dm + 2 * 2 * BN * 4 + 127) & ~127;
+    static constexpr size_t total = (size_t)sc + 2 * kScSlotBytes + 1024;
 };
 
 struct Params {
@@ -122,7 +118,6 @@ struct Params {
     int out_f32;
     int* err;
     int splits;            // K slices per output tile (1 = no split)
-    int sc_ring;           // 1: per-group dx/S arrive by TMA in a shared ring
     int tiles_n;           // output tiles along N
     int units;             // tiles * splits work units (CTAs loop over them)
     int* counters;         // [tiles] arrival counters (split > 1), zeroed before launch
@@ -216,13 +211,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* drain = tempty + NPAIR;        // final MMA completion
     uint64_t* scfull = drain + 1;            // a group's dx/S landed in its slot
     uint64_t* scempty = scfull + 2;          // the epilogue has read the slot
+    uint64_t* dmfull = scempty + 2;          // a group's d, m written to their slot
+    uint64_t* dmfree = dmfull + 2;           // every epilogue warp has read the slot
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Smem::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
     volatile int* last_flag = abort_flag + 1;
-    float* d_s = reinterpret_cast<float*>(smem + Smem::dm);
+    float* dm_s = reinterpret_cast<float*>(smem + Smem::dm);  // [2][2][BN]
     const int G = p.K / 256;
-    float* m_s = d_s + G * BN;
-    uint8_t* sc = smem + Smem::sc(G);
+    uint8_t* sc = smem + Smem::sc;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -253,6 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 2; ++i) {
             w4::mbar_init(&scfull[i], 1);
             w4::mbar_init(&scempty[i], kEpiWarps);
+            w4::mbar_init(&dmfull[i], kEpiWarps);
+            w4::mbar_init(&dmfree[i], kEpiWarps);
         }
         *abort_flag = 0;
         w4::fence_mbar_init();
@@ -278,16 +276,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 48;");
         if (warp == 0) {
             // ---------------- TMA producer ----------------
             if (w4::elect_one()) {
                 w4::prefetch_tmap(&tm_a);
                 w4::prefetch_tmap(&tm_b);
-                if (p.sc_ring) {
-                    w4::prefetch_tmap(&tm_dx);
-                    w4::prefetch_tmap(&tm_s);
-                }
+                w4::prefetch_tmap(&tm_dx);
+                w4::prefetch_tmap(&tm_s);
                 int it = 0;  // global stage counter
                 int gi = 0;  // groups whose scales were issued
                 bool ok = true;
@@ -295,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     int tmi, tni, gb, ge;
                     unit_of(u, tmi, tni, gb, ge);
                     for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
-                        if (p.sc_ring && (kg & 1) == 0) {
+                        if ((kg & 1) == 0) {
                             // the group's dx and S for the tile's 128 tokens, ahead of
                             // its first stage (rows past M are zero-filled)
                             const int slot = gi & 1;
@@ -427,38 +423,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue (warps 4..11) ----------------
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
         const int et = threadIdx.x - 128;           // 0..255
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
         const int cs = (warp - 4) >> 2;             // column slice: kEpiCols weight rows
         const int row = quarter * 32 + lane;        // token row within the tile
-        const int B = p.K / KB;
         const uint32_t tm_row =
             tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cs * kEpiCols);
 
         int it = 0;
-        int gi = 0;  // groups started (the scale ring's slot sequence)
+        int gi = 0;  // groups started (the slot sequence of both per-group rings)
         bool ok = true;
+        // d and m travel per group through a two-slot ring: thread et owns one
+        // value (d if et < 128, else m) of weight row (et & 127) of the tile; it
+        // loads the next group's value at a group's start and writes it to the
+        // other slot at the group's end.
+        auto dm_value = [&](int n0v, int gv) -> float {
+            const int n = n0v + (et & (BN - 1));
+            const __half* src = (et >> 7) ? p.m : p.d;
+            return n < p.N ? __half2float(src[(size_t)n * G + gv]) : 0.0f;
+        };
+        if (blockIdx.x < p.units) {
+            int tmi0, tni0, gb0, ge0;
+            unit_of(blockIdx.x, tmi0, tni0, gb0, ge0);
+            dm_s[et] = dm_value(tni0 * BN, gb0);  // slot 0 ([d, m][BN]): first group
+            __syncwarp();
+            if (lane == 0) w4::mbar_arrive(&dmfull[0]);
+        }
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             int tmi, tni, g_begin, g_end;
             unit_of(u, tmi, tni, g_begin, g_end);
             const int n0 = tni * BN;
             const int t = tmi * BM + row;
             const bool t_live = t < p.M;
-            // this tile's d and m, fp32 [g][n]; rows past N -> 0
-            asm volatile("bar.sync 1, 256;" ::: "memory");  // previous unit done with them
-            for (int i = et; i < BN * (g_end - g_begin); i += 256) {
-                const int r = i / (g_end - g_begin), g = g_begin + (i - r * (g_end - g_begin));
-                const int n = n0 + r;
-                float dv = 0.0f, mv = 0.0f;
-                if (n < p.N) {
-                    dv = __half2float(p.d[(size_t)n * G + g]);
-                    mv = __half2float(p.m[(size_t)n * G + g]);
-                }
-                d_s[g * BN + r] = dv;
-                m_s[g * BN + r] = mv;
-            }
-            asm volatile("bar.sync 1, 256;" ::: "memory");
 
             float acc[kEpiCols], yv[kEpiCols];
 #pragma unroll
@@ -470,9 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             float cf[8];  // per-block coefficients of the current group, times 2^e
 #pragma unroll
             for (int i = 0; i < 8; ++i) cf[i] = 0.0f;
-            const float* dx_row = p.dx + (size_t)(t_live ? t : 0) * B;
-            const int32_t* s_row = p.S + (size_t)(t_live ? t : 0) * B;
             const int ksteps = (g_end - g_begin) * 2;
+            int gcur = 0;           // this group's index in the slot sequence
+            float dm_next = 0.0f;   // this thread's d or m value of the next group
+            bool has_next = false;
             for (int ks = 0; ks < ksteps && ok; ++ks, ++it) {
                 const int g = g_begin + (ks >> 1);  // global group index
                 const bool first_half = (ks & 1) == 0;
@@ -486,10 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i) dxg[i] = 0.0f;
                     tmin = 0.0f;
-                    float4 sa4[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-                    int4 ss4[2] = {make_int4(0, 0, 0, 0), make_int4(0, 0, 0, 0)};
-                    if (p.sc_ring) {
-                        // this token's 8 scales and sums, brought in by TMA
+                    float4 sa4[2];
+                    int4 ss4[2];
+                    {
+                        // this token's 8 scales and sums, brought in by TMA (zero past M)
                         const int slot = gi & 1;
                         if (!w4::mbar_wait(&scfull[slot], (uint32_t)(gi >> 1) & 1u, abort_flag,
                                            p.err)) {
@@ -504,14 +502,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                             reinterpret_cast<const int4*>(src + Smem::kScSlotBytes / 2)[2 * row + 1];
                         __syncwarp();
                         if (lane == 0) w4::mbar_arrive(&scempty[slot]);
-                    } else if (t_live) {
-#pragma unroll
-                        for (int h4 = 0; h4 < 2; ++h4) {
-                            sa4[h4] = __ldg(reinterpret_cast<const float4*>(dx_row + g * 8) + h4);
-                            ss4[h4] = __ldg(reinterpret_cast<const int4*>(s_row + g * 8) + h4);
-                        }
                     }
+                    gcur = gi;
                     ++gi;
+                    // the next group's d or m, a whole group ahead of its use
+                    if (g + 1 < g_end) {
+                        has_next = true;
+                        dm_next = dm_value(n0, g + 1);
+                    } else if (u + (int)gridDim.x < p.units) {
+                        int tmi2, tni2, gb2, ge2;
+                        unit_of(u + gridDim.x, tmi2, tni2, gb2, ge2);
+                        has_next = true;
+                        dm_next = dm_value(tni2 * BN, gb2);
+                    } else {
+                        has_next = false;
+                    }
                     {
 #pragma unroll
                         for (int h4 = 0; h4 < 2; ++h4) {
@@ -578,8 +583,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (ok && !first_half) {
                     // y += d * (acc * 2^(149-e) - 2^17 * sum_{r<4} dx_r) + m * sum dx S
-                    const float4* dg = reinterpret_cast<const float4*>(d_s + g * BN + cs * kEpiCols);
-                    const float4* mg = reinterpret_cast<const float4*>(m_s + g * BN + cs * kEpiCols);
+                    const int slot = gcur & 1;
+                    if (!w4::mbar_wait(&dmfull[slot], (uint32_t)(gcur >> 1) & 1u, abort_flag,
+                                       p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const float* ds = dm_s + slot * 2 * BN;
+                    const float4* dg = reinterpret_cast<const float4*>(ds + cs * kEpiCols);
+                    const float4* mg = reinterpret_cast<const float4*>(ds + BN + cs * kEpiCols);
 #pragma unroll
                     for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
                         const float4 dv = dg[c4], mv = mg[c4];
@@ -592,6 +604,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                             yv[c] = fmaf(dvv[e4], av, fmaf(mvv[e4], tmin, yv[c]));
                             acc[c] = 0.0f;
                         }
+                    }
+                    __syncwarp();
+                    if (lane == 0) w4::mbar_arrive(&dmfree[slot]);
+                    if (has_next) {
+                        // the other slot was last read at the previous group's end
+                        const int nslot = slot ^ 1;
+                        if (gcur >= 1 &&
+                            !w4::mbar_wait(&dmfree[nslot], (uint32_t)((gcur - 1) >> 1) & 1u,
+                                           abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        dm_s[nslot * 2 * BN + et] = dm_next;
+                        __syncwarp();
+                        if (lane == 0) w4::mbar_arrive(&dmfull[nslot]);
                     }
                 }
             }
@@ -747,6 +774,7 @@ bool make_map_4b(CUtensorMap* map, const void* base, CUtensorMapDataType type, u
 
 // Usable dynamic shared memory per CTA on sm_100.
 constexpr size_t kSmemMax = 227 * 1024;
+static_assert(Smem::total <= kSmemMax, "shared memory layout exceeds one CTA's allotment");
 
 // K slices per output tile.  Cost model in units of one 256-group of MMA work
 // per CTA: waves(tiles * S over the SMs) * (groups per slice + fixed cost of a
@@ -819,29 +847,21 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
                      CU_TENSOR_MAP_SWIZZLE_NONE))
         return W4_ERR_CUDA;
 
-    const int G = (int)(K / 256);
-    // the scale ring when it fits next to d and m (every K up to 42 groups)
-    const bool ring = Smem::total(G, true) <= kSmemMax;
-    const size_t smem = Smem::total(G, ring);
+    const size_t smem = Smem::total;
+    // dx and S are [M][K/32]: row stride K/8 bytes (a multiple of 16), box 8 x 128
     CUtensorMap mdx, ms;
-    if (ring) {
-        // dx and S are [M][K/32]: row stride K/8 bytes (a multiple of 16), box 8 x 128
-        if (!make_map_4b(&mdx, dx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)K / 32,
-                         (uint64_t)M, 8, BM) ||
-            !make_map_4b(&ms, bsum, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)K / 32, (uint64_t)M,
-                         8, BM))
-            return W4_ERR_CUDA;
-    } else {
-        mdx = ma;  // unused by the kernel
-        ms = ma;
-    }
+    if (!make_map_4b(&mdx, dx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, (uint64_t)K / 32, (uint64_t)M, 8,
+                     BM) ||
+        !make_map_4b(&ms, bsum, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)K / 32, (uint64_t)M, 8,
+                     BM))
+        return W4_ERR_CUDA;
     static thread_local int attr_dev = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return w4::cuda_fail(e);
     if (attr_dev != dev) {
         e = cudaFuncSetAttribute(w4a8_mmq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemMax);
+                                 (int)Smem::total);
         if (e != cudaSuccess) return w4::cuda_fail(e);
         attr_dev = dev;
     }
@@ -857,7 +877,6 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     prm.out_f32 = out_dtype == W4_OUT_F32;
     prm.err = err;
     prm.splits = splits;
-    prm.sc_ring = ring ? 1 : 0;
     prm.counters = nullptr;
     prm.partials = nullptr;
     if (splits > 1) {
