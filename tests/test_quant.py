@@ -53,3 +53,25 @@ def test_quant_special_blocks(torch, w4, orc):
 def test_quant_bit_exact_full_size(torch, w4, orc, M, K):
     _check(torch, w4, orc, synth.outlier_activations(M, K, seed=synth.act_seed(
         synth.CONFIG_MMQ, 0 if K == 2560 else 1)))
+
+
+def test_quant_near_half_integer_quotients(torch, w4, orc):
+    # Every block holds its amax (which fixes dx = amax / 127) and 31 bf16
+    # values on or next to half-integer multiples (k + 1/2) dx: the quotients
+    # whose rounding to an integer depends on the last bit of x / dx.  The
+    # codes must equal rint(fl(x / dx)) exactly.
+    rng = np.random.default_rng(31)
+    nblk = 4096
+    x = np.zeros((nblk, 32), np.float32)
+    amax = synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(
+        (2.0 ** rng.uniform(-20, 20, nblk)).astype(np.float32)))
+    dx = (amax / np.float32(127.0)).astype(np.float32)
+    k = rng.integers(0, 127, (nblk, 31)).astype(np.float64)
+    target = ((k + 0.5) * dx[:, None].astype(np.float64)).astype(np.float32)
+    bits = synth.f32_to_bf16_bits(target).astype(np.int32)
+    bits += rng.integers(-2, 3, bits.shape)            # the nearest bf16 values and neighbours
+    vals = synth.bf16_bits_to_f32(bits.astype(np.uint16))
+    vals = np.minimum(np.abs(vals), amax[:, None]) * np.where(rng.random(vals.shape) < 0.5, -1, 1)
+    x[:, 0] = amax
+    x[:, 1:] = vals
+    _check(torch, w4, orc, synth.f32_to_bf16_bits(x.reshape(64, -1)))

@@ -12,6 +12,17 @@
 // block and reduce amax and S with two xor-shuffles.  K % 32 == 0 means a
 // block never straddles a row, so the flattened [M][K] array is processed as
 // one stream.
+//
+// Division.  A full IEEE division per element made the kernel issue-bound.
+// All 32 elements of a block share the divisor dx, so each element's quotient
+// is formed by Markstein's correction of a reciprocal product (P. Markstein,
+// IBM J. Res. Dev. 34(1), 1990; also Cornea, Harrison and Tang, "Scientific
+// Computing on Itanium-based Systems", 2002): r = RN(1/dx) once per block,
+// q0 = x r, e = x - q0 dx (one FMA, exact), q = q0 + e r.  q is within an
+// ulp of the IEEE quotient fl(x / dx) (|q| <= ~127 here, ulp <= 2^-16), so
+// rint(q) = rint(fl(x / dx)) whenever q is farther than 2^-14 from a
+// half-integer; elements that land closer (rare) take the IEEE division
+// itself.  The codes therefore equal clamp(rint(fl(x / dx))) exactly.
 #include "common.cuh"
 
 namespace {
@@ -42,9 +53,13 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __rest
         int sum = 0;
         uint32_t packed[2] = {0u, 0u};
         if (amax != 0.0f) {
+            const float rcp = __frcp_rn(scale);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                float qf = rintf(__fdiv_rn(f[j], scale));
+                const float q0 = f[j] * rcp;
+                const float q = fmaf(fmaf(-q0, scale, f[j]), rcp, q0);
+                float qf = rintf(q);
+                if (fabsf(fabsf(q - qf) - 0.5f) < 0x1p-14f) qf = rintf(__fdiv_rn(f[j], scale));
                 qf = fminf(fmaxf(qf, -127.0f), 127.0f);
                 const int qi = (int)qf;
                 sum += qi;
