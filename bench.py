@@ -615,13 +615,7 @@ def run_ours(args):
             "ms_per_step": round(elapsed_max / args.steps * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "u4 codes x bf16 (fp32 accumulate)", "data": "synthetic",
-            "config": {"workload": "batch-1 decode GEMV sweep, W4-G256, (N,K) = "
-                                   "(6144,2560) (2560,4096) (19456,2560) (2560,9728) "
-                                   "(151936,2560), M=1, bf16 out",
-                       "global_batch": world, "seq_len": 1,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2: two 253 MB weight sets alternate",
-                       "launch": "each step replays a CUDA graph of the five GEMVs"},
+            "config": run_config(world),
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches,
             "clocks": clk.summary(), "cpu_baseline": cpu,
         }
@@ -671,6 +665,17 @@ def cpu_baseline(seconds: float = 15.0, rows_per_shape: int = 2048) -> dict:
                       f"{reps} passes, {dt:.1f} s"}
 
 
+def run_config(world: int) -> dict:
+    """The workload both arms report on."""
+    return {"workload": "batch-1 decode GEMV sweep, W4-G256, (N,K) = "
+                        "(6144,2560) (2560,4096) (19456,2560) (2560,9728) "
+                        "(151936,2560), M=1, bf16 out",
+            "global_batch": world, "seq_len": 1,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: two 253 MB weight sets alternate",
+            "launch": "each step replays a CUDA graph of the five GEMVs"}
+
+
 def run_reference(args):
     world, rank, local = dist_env()
     if rank != 0:
@@ -695,8 +700,7 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "batch-1 decode GEMV sweep, W4-G256 (CPU oracle sample)",
-                   "global_batch": 1, "seq_len": 1, "parallelism": "cpu"},
+        "config": run_config(world),
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": o.num_threads(),
                          "kind": "oracle", "sample": sample_desc},
         "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
