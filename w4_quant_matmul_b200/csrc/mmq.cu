@@ -14,7 +14,9 @@
 // the whole launch.  K advances in stages of 128 (four 32-element activation
 // blocks); two stages make one 256-group.
 //   warp 0      TMA producer: the qa tile (128 x 128 B, 128B-swizzled) and the
-//               packed code tile (128 rows x 64 B) into a 4-stage ring.
+//               packed code tile (128 rows x 64 B) into a 4-stage ring, and,
+//               ahead of each 256-group, that group's dx and S for the tile's
+//               128 tokens (8 x 128 boxes of fp32 / int32) into a 2-slot ring.
 //   warp 1      allocates 512 TMEM columns = four 128-column block buffers;
 //               one lane issues, per 32-block, a tcgen05.mma.kind::i8 (M=128,
 //               N=128, K=32; A = qa as s8, B = the codes as u8) into the
@@ -26,7 +28,11 @@
 //   warps 4-11  epilogue: each thread owns one token row (its TMEM lane) and 64
 //               weight rows; per buffer pair it waits once, reads both blocks'
 //               words and releases the pair; the thread that sees a stage's
-//               last pair also frees that stage's shared-memory operands.
+//               last pair also frees that stage's shared-memory operands.  d
+//               and m move per group through a 2-slot shared ring: each of the
+//               256 epilogue threads loads one of the tile's next-group values
+//               a group ahead and writes it at the group's end.  Shared memory
+//               (~190 KB) does not depend on K.
 //
 // On B200 the tensor pipe runs MMAs and commits one after another, and a
 // commit costs about as much as 1.5 of these MMAs (measured), so commits are
