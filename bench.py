@@ -299,7 +299,7 @@ def time_gemv_sweep(torch, w4, wl, M, steps, warmup, stream):
     return elapsed, per, steps * len(SHAPES)
 
 
-def time_w4a8_gemv(torch, w4, wl, M, steps, stream):
+def time_w4a8_gemv(torch, w4, wl, M, steps, stream, fused=False):
     """Keep-quant decode GEMV (int8 activation blocks from q8_quantize_act,
     quantised once outside the timed launches): per-shape mean ms, each launch
     its own CUDA graph between events, shapes in sweep order so the lm_head
@@ -310,6 +310,10 @@ def time_w4a8_gemv(torch, w4, wl, M, steps, stream):
 
     def run(c, s):
         codes, d, m = wl.weights[c][s]
+        if fused:  # quantiser folded into the GEMV: bf16 x in
+            w4.w4a8_gemv_bf16(codes, d, m, xs[s], out_dtype=torch.bfloat16, y=ys[s],
+                              stream=stream)
+            return
         qa, dx, S = acts[s]
         w4.w4a8_gemv(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=ys[s], stream=stream)
 
@@ -587,6 +591,14 @@ def run_ours(args):
             extras[f"w4a8_gemv_m{M}"] = [
                 {"N": n, "K": k, "us": round(ms * 1e3, 2),
                  "gbs": round(w4a8_gemv_bytes(n, k, M) / (ms / 1e3) / 1e9, 1),
+                 "tok_per_s": round(M / (ms / 1e3), 1)}
+                for (n, k), ms in zip(SHAPES, per)]
+            # the same product from bf16 x, quantiser folded in (algorithmic
+            # bytes: the bf16 GEMV's)
+            per = time_w4a8_gemv(torch, w4, wl, M, max(3, args.steps // 2), stream, fused=True)
+            extras[f"w4a8_gemv_bf16_m{M}"] = [
+                {"N": n, "K": k, "us": round(ms * 1e3, 2),
+                 "gbs": round(gemv_bytes(n, k, M) / (ms / 1e3) / 1e9, 1),
                  "tok_per_s": round(M / (ms / 1e3), 1)}
                 for (n, k), ms in zip(SHAPES, per)]
         del wl

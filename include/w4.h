@@ -133,6 +133,17 @@ int w4a8_gemv(const uint8_t *codes, const uint16_t *d_f16,
               const float *dx, const int32_t *bsum, int M, void *y,
               int out_dtype, void *stream);
 
+/* w4a8_gemv with the activation quantiser folded in: takes bf16 x [M][K] and
+ * quantises each 32-element block inside the GEMV, with the arithmetic of
+ * q8_quantize_act, so y is bit-identical to q8_quantize_act followed by
+ * w4a8_gemv, without the second launch or the int8 blocks' round trip
+ * through memory (the "fold the quantiser into its neighbour" next step of
+ * the decode path).  Arguments and errors as w4_gemv. */
+int w4a8_gemv_bf16(const uint8_t *codes, const uint16_t *d_f16,
+                   const uint16_t *m_f16, int64_t N, int64_t K,
+                   const uint16_t *x_bf16, int M, void *y, int out_dtype,
+                   void *stream);
+
 /* Quantise bf16 activations to int8 per block of 32 (the article's
  * "pre-quantise prefill activations to the Q8_1 MMQ layout"), with the
  * reading adopted for the unprinted rule:

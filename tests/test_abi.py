@@ -29,7 +29,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for expected in ["w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "w4a8_gemv",
-                     "q8_quantize_act",
+                     "w4a8_gemv_bf16", "q8_quantize_act",
                      "w4a8_mmq", "w4a8_mmq_workspace_size", "w4_status_string",
                      "w4_abi_version", "w4_last_cuda_error", "w4_check_device_error"]:
         assert expected in names

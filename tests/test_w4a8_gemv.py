@@ -151,3 +151,24 @@ def test_rejects_bad_arguments(torch, w4):
     with pytest.raises(w4.W4Error):
         w4.w4a8_gemv(codes, d, d, qa, dx, S)   # M = 9
     w4.w4_check_device_error()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 6144, 2560), (4, 300, 9728), (8, 151936, 2560)])
+def test_fused_quantiser_is_bit_identical(torch, w4, orc, M, N, K):
+    # w4a8_gemv_bf16 (quantiser folded in) == q8_quantize_act + w4a8_gemv, bit
+    # for bit, on both GEMV kernels (the last shape takes the row kernel)
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=N + K)
+    x = synth.outlier_activations(M, K, seed=M + 40)
+    dc, dd, dm = (torch.from_numpy(codes).cuda(), _dev_u16(torch, d, torch.float16),
+                  _dev_u16(torch, m, torch.float16))
+    xd = _dev_u16(torch, x, torch.bfloat16)
+    fused = w4.w4a8_gemv_bf16(dc, dd, dm, xd, out_dtype=torch.float32)
+    qa, dx, S = w4.q8_quantize_act(xd)
+    two_step = w4.w4a8_gemv(dc, dd, dm, qa, dx, S, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(fused.view(torch.int32), two_step.view(torch.int32))
+    rows = parity.sample_rows(N, count=64)
+    qa_o, dx_o, S_o = orc.q8_quantize(x)
+    ref = np.concatenate([orc.mmq(codes, d, m, qa_o, dx_o, S_o, rows=(int(r), int(r) + 1))
+                          for r in rows], axis=1)
+    parity.assert_f32_gate(fused.cpu().numpy()[:, rows], ref, f"fused M{M} {N}x{K}")

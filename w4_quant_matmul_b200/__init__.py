@@ -12,6 +12,7 @@ Entry points (same names as the C ABI):
     w4_unpack(codes, K)                     -> q
     w4_gemv(codes, d, m, x, out_dtype)      -> y
     w4a8_gemv(codes, d, m, qa, dx, bsum, out_dtype) -> y   (int8 activations, M <= 8)
+    w4a8_gemv_bf16(codes, d, m, x, out_dtype) -> y   (x quantised inside, M <= 8)
     q8_quantize_act(x)                      -> qa, dx, bsum
     w4a8_mmq(codes, d, m, qa, dx, bsum, out_dtype) -> y
     w4a8_mmq_static(codes, d, m, qa, dx, bsum, out_dtype) -> y   (no workspace)
@@ -24,6 +25,7 @@ from ._lib import (LibraryMissing, W4_OK, W4_OUT_BF16, W4_OUT_F32, load, status_
 
 __all__ = [
     "W4Error", "LibraryMissing", "w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "w4a8_gemv",
+    "w4a8_gemv_bf16",
     "q8_quantize_act", "w4a8_mmq", "w4a8_mmq_static", "w4a8_mmq_workspace_size",
     "w4_check_device_error",
     "w4_abi_version", "lib",
@@ -186,6 +188,27 @@ def w4a8_gemv(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, stream=None):
                         device=qa.device)
     _check(load().w4a8_gemv(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(qa), _ptr(dx), _ptr(bsum),
                             M, _ptr(y), oc, _stream(stream)), "w4a8_gemv")
+    return y
+
+
+def w4a8_gemv_bf16(codes, d, m, x, out_dtype=None, y=None, stream=None):
+    """w4a8_gemv with the quantiser folded in: bf16 x[M,K] (1 <= M <= 8) is
+    quantised to int8 blocks inside the kernel; bit-identical to
+    q8_quantize_act followed by w4a8_gemv."""
+    torch = _torch()
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    _need(codes, torch.uint8, "codes")
+    _need(d, torch.float16, "d")
+    _need(m, torch.float16, "m")
+    _need(x, torch.bfloat16, "x")
+    N = codes.shape[0]
+    M, K = x.shape
+    oc = _out_code(out_dtype)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32 if oc == W4_OUT_F32 else torch.bfloat16,
+                        device=x.device)
+    _check(load().w4a8_gemv_bf16(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x), M, _ptr(y), oc,
+                                 _stream(stream)), "w4a8_gemv_bf16")
     return y
 
 

@@ -37,6 +37,7 @@ SIGNATURES = {
     "w4_unpack": ([_P, _I64, _I64, _P, _P], _INT),
     "w4_gemv": ([_P, _P, _P, _I64, _I64, _P, _INT, _P, _INT, _P], _INT),
     "w4a8_gemv": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _INT, _P, _INT, _P], _INT),
+    "w4a8_gemv_bf16": ([_P, _P, _P, _I64, _I64, _P, _INT, _P, _INT, _P], _INT),
     "q8_quantize_act": ([_P, _I64, _I64, _P, _P, _P, _P], _INT),
     "w4a8_mmq_workspace_size": ([_I64, _I64, _I64], ctypes.c_size_t),
     "w4a8_mmq": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P, ctypes.c_size_t, _P],

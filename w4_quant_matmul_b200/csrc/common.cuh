@@ -148,4 +148,19 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
+// The int8 code of one activation, x -> clamp(rint(fl(x / dx)), -127, 127),
+// given the block's dx != 0 and rcp = RN(1 / dx).  Markstein's correction of
+// the reciprocal product (P. Markstein, IBM J. Res. Dev. 1990): q = q0 +
+// (x - q0 dx) rcp is within an ulp of fl(x / dx), so its rounding to an
+// integer is that of fl(x / dx) unless q lies within 2^-14 of a half-integer,
+// where the IEEE division itself decides.  Shared by the quantiser and the
+// GEMV that quantises its activations in place, so both give the same codes.
+__device__ __forceinline__ int q8_code(float x, float dx, float rcp) {
+    const float q0 = x * rcp;
+    const float q = fmaf(fmaf(-q0, dx, x), rcp, q0);
+    float qf = rintf(q);
+    if (fabsf(fabsf(q - qf) - 0.5f) < 0x1p-14f) qf = rintf(__fdiv_rn(x, dx));
+    return (int)fminf(fmaxf(qf, -127.0f), 127.0f);
+}
+
 }  // namespace w4

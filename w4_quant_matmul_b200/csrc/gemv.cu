@@ -62,6 +62,14 @@ constexpr int kThreads = 256;
 constexpr int kHalfWarps = kThreads / 16;
 constexpr int kSmemBudget = 200 * 1024;
 
+// Activations: bf16 x [M][K] as 16-bit fixed-point words (kActBf16); int8
+// blocks of 32 with their scales and sums (kActInt8: qa [M][K], dx and S
+// [M][K/32]); or bf16 x [M][K] quantised to those int8 blocks in shared
+// memory, with the quantiser's arithmetic (kActBf16ToInt8).
+constexpr int kActBf16 = 0;
+constexpr int kActInt8 = 1;
+constexpr int kActBf16ToInt8 = 2;
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
     uint4 r;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -119,7 +127,7 @@ __device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __res
     }
 }
 
-template <int M, int RH, int U, bool A8>
+template <int M, int RH, int U, int AM>
 __device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4* __restrict__ xq,
                                               const float* __restrict__ sx,
                                               const float* __restrict__ inv, int C, int c0,
@@ -153,7 +161,7 @@ __device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4
                 for (int t = 0; t < M; ++t) {
                     ah[t][i] = __dp4a((int)lo, (int)xv[t].x, ah[t][i]);
                     ah[t][i] = __dp4a((int)hi, (int)xv[t].y, ah[t][i]);
-                    if constexpr (!A8) {
+                    if constexpr (AM == kActBf16) {
                         al[t][i] = (int)__dp4a(lo, xv[t].z, (unsigned)al[t][i]);
                         al[t][i] = (int)__dp4a(hi, xv[t].w, (unsigned)al[t][i]);
                     }
@@ -167,8 +175,8 @@ __device__ __forceinline__ void consume_batch(const Batch<RH, U>& b, const uint4
             for (int i = 0; i < RH; ++i) {
                 const float dd = __half2float(__ushort_as_half((unsigned short)(b.dm[u][i] & 0xFFFFu)));
                 const float mm = __half2float(__ushort_as_half((unsigned short)(b.dm[u][i] >> 16)));
-                // A8: the exact block dot P times dx; else (sum q X) / sigma
-                const float qx = (A8 ? (float)ah[t][i] : (float)(ah[t][i] * 256 + al[t][i])) * iv;
+                // int8 blocks: the exact block dot P times dx; else (sum q X) / sigma
+                const float qx = (AM != kActBf16 ? (float)ah[t][i] : (float)(ah[t][i] * 256 + al[t][i])) * iv;
                 yacc[t][i] = fmaf(dd, qx, fmaf(mm, s, yacc[t][i]));
             }
         }
@@ -228,8 +236,7 @@ __device__ __forceinline__ void stage_quarter(uint4 raw, bool live, uint4* __res
     }
 }
 
-// Activations: bf16 x [M][K] (A8 = false), or int8 blocks of 32 with their
-// scales and sums (A8 = true: qa [M][K], dx and S [M][K/32]).
+// Activation forms (the Act pointers below).
 struct Act {
     const void* x;
     const float* dx;
@@ -257,6 +264,50 @@ __device__ __forceinline__ void stage_block_a8(const Act& a, int C, int t, int c
     inv[t * C + c] = dxv;
 }
 
+// One bf16 activation block (32 values of token t, chunk c) quantised to int8
+// exactly as q8_quantize_act does (dx = fl(amax / 127), codes by q8_code,
+// S = sum of codes), then staged like stage_block_a8.
+__device__ __forceinline__ void stage_block_q8x(const Act& a, int C, int t, int c,
+                                                uint4* __restrict__ xq, float* __restrict__ sx,
+                                                float* __restrict__ inv) {
+    const uint4* src = reinterpret_cast<const uint4*>(
+        reinterpret_cast<const uint16_t*>(a.x) + ((size_t)t * C + c) * 32);
+    uint32_t raw[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldg(src + i);
+        raw[4 * i] = v.x;
+        raw[4 * i + 1] = v.y;
+        raw[4 * i + 2] = v.z;
+        raw[4 * i + 3] = v.w;
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(raw[i])), fabsf(bf16_hi(raw[i]))));
+    const float dxv = __fdiv_rn(amax, 127.0f);
+    uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // the 32 codes, 4 per word
+    int S = 0;
+    if (amax != 0.0f) {
+        const float rcp = __frcp_rn(dxv);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int q0 = w4::q8_code(bf16_lo(raw[i]), dxv, rcp);
+            const int q1 = w4::q8_code(bf16_hi(raw[i]), dxv, rcp);
+            S += q0 + q1;
+            w[i >> 1] |= (((uint32_t)q0 & 0xFFu) | (((uint32_t)q1 & 0xFFu) << 8)) << (16 * (i & 1));
+        }
+    }
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi)
+        xq[((size_t)t * 4 + wi) * C + c] =
+            make_uint4(__byte_perm(w[2 * wi], w[2 * wi + 1], 0x6420),
+                       __byte_perm(w[2 * wi], w[2 * wi + 1], 0x7531), 0u, 0u);
+    const float dxs = amax == 0.0f ? 0.0f : dxv;
+    sx[t * C + c] = dxs * (float)S;
+    inv[t * C + c] = dxs;
+}
+
 // Resident CTAs per SM the register allocation is sized for: small M needs
 // many warps in flight to cover HBM latency; large M needs the registers.
 template <int M>
@@ -264,7 +315,7 @@ struct MinCtas {
     static constexpr int value = M == 1 ? 3 : (M <= 4 ? 2 : 1);
 };
 
-template <int M, int RH, int U, bool A8>
+template <int M, int RH, int U, int AM>
 __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
     int N, int K, int KS, const Act act, void* __restrict__ y, int out_f32) {
@@ -308,9 +359,12 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
     pdl_wait();
 
     // ---- activation words, chunk sums and scales, once per CTA ----
-    if constexpr (A8) {
+    if constexpr (AM == kActInt8) {
         for (int v = threadIdx.x; v < M * C; v += kThreads)
             stage_block_a8(act, C, v / C, v - (v / C) * C, xq, sx, inv);
+    } else if constexpr (AM == kActBf16ToInt8) {
+        for (int v = threadIdx.x; v < M * C; v += kThreads)
+            stage_block_q8x(act, C, v / C, v - (v / C) * C, xq, sx, inv);
     } else {
         const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
         for (int base = 0; base < nq; base += kThreads) {
@@ -340,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
         if (active) {
             for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
                 if (c0 != cs + j) load_batch(bt, codes, d, m, rows, row_bytes, G, c0, ce);
-                consume_batch<M, RH, U, A8>(bt, xq, sx, inv, C, c0, ce, yacc);
+                consume_batch<M, RH, U, AM>(bt, xq, sx, inv, C, c0, ce, yacc);
             }
         }
         // reduce the 16 lanes of the half-warp (xor < 16 stays inside it)
@@ -417,11 +471,11 @@ size_t smem_bytes(int M, int C, int KS, int RH) {
            (KS > 1 ? (size_t)KS * rows_per_cta * M * 4 : 0);
 }
 
-template <int M, int RH, bool A8>
+template <int M, int RH, int AM>
 int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K, int KS,
            const Act& x, void* y, int out_f32, cudaStream_t st) {
     constexpr int U = 8 / RH;
-    auto kern = w4_gemv_rows_kernel<M, RH, U, A8>;
+    auto kern = w4_gemv_rows_kernel<M, RH, U, AM>;
     const int C = K / 32;
     const size_t smem = smem_bytes(M, C, KS, RH);
     // Per-instantiation cache: one device, a few shared-memory sizes.
@@ -486,7 +540,7 @@ void pick_split(int N, int C, int sms, int* rh, int* ks) {
     *ks = k;
 }
 
-template <int M, bool A8>
+template <int M, int AM>
 int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                const Act& x, void* y, int out_f32, cudaStream_t st) {
     int rh, ks;
@@ -494,10 +548,10 @@ int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N
     if (M >= 4 && rh > 2) rh = 2;  // register budget: M * RH accumulators twice
     if (smem_bytes(M, K / 32, ks, rh) > (size_t)kSmemBudget) ks = 1;
     if constexpr (M < 4) {
-        if (rh == 4) return launch_rows<M, 4, A8>(codes, d, m, N, K, ks, x, y, out_f32, st);
+        if (rh == 4) return launch_rows<M, 4, AM>(codes, d, m, N, K, ks, x, y, out_f32, st);
     }
-    if (rh >= 2) return launch_rows<M, 2, A8>(codes, d, m, N, K, ks, x, y, out_f32, st);
-    return launch_rows<M, 1, A8>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    if (rh >= 2) return launch_rows<M, 2, AM>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    return launch_rows<M, 1, AM>(codes, d, m, N, K, ks, x, y, out_f32, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -537,7 +591,7 @@ struct RingMinCtas {
     static constexpr int value = M <= 4 ? 2 : 1;
 };
 
-template <int M, bool A8>
+template <int M, int AM>
 __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_ring_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
     int N, int K, int stages, int rows_per_cta, const Act act, void* __restrict__ y, int out_f32,
@@ -612,9 +666,12 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
     // activation words, chunk sums and scales, once per CTA; each thread issues
     // up to four 16-byte loads before converting any
     constexpr int kCons = 32 * kRingWarps;
-    if constexpr (A8) {
+    if constexpr (AM == kActInt8) {
         for (int v = threadIdx.x; v < M * C; v += kCons)
             stage_block_a8(act, C, v / C, v - (v / C) * C, xq, sx, inv);
+    } else if constexpr (AM == kActBf16ToInt8) {
+        for (int v = threadIdx.x; v < M * C; v += kCons)
+            stage_block_q8x(act, C, v / C, v - (v / C) * C, xq, sx, inv);
     } else {
         const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
         for (int base = 0; base < nq; base += 4 * kCons) {
@@ -713,7 +770,7 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
                         const uint4 xv = xq[((size_t)t * 4 + wi) * C + c];
                         ah[t] = __dp4a((int)lo, (int)xv.x, ah[t]);
                         ah[t] = __dp4a((int)hi, (int)xv.y, ah[t]);
-                        if constexpr (!A8) {
+                        if constexpr (AM == kActBf16) {
                             al[t] = (int)__dp4a(lo, xv.z, (unsigned)al[t]);
                             al[t] = (int)__dp4a(hi, xv.w, (unsigned)al[t]);
                         }
@@ -724,7 +781,7 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
 #pragma unroll
                 for (int t = 0; t < M; ++t) {
                     const float qx =
-                        (A8 ? (float)ah[t] : (float)(ah[t] * 256 + al[t])) * inv[t * C + c];
+                        (AM != kActBf16 ? (float)ah[t] : (float)(ah[t] * 256 + al[t])) * inv[t * C + c];
                     const float v = fmaf(dd, qx, fmaf(mm, sx[t * C + c], yacc[t]));
                     yacc[t] = live ? v : yacc[t];
                 }
@@ -776,10 +833,10 @@ Plan plan_for(int M, int C) {
     return p;
 }
 
-template <int M, bool A8>
+template <int M, int AM>
 int launch_ring(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                 const Act& x, void* y, int out_f32, cudaStream_t st) {
-    auto kern = w4_gemv_ring_kernel<M, A8>;
+    auto kern = w4_gemv_ring_kernel<M, AM>;
     const Plan pl = plan_for(M, K / 32);  // per_sm matches RingMinCtas<M>
     if (pl.stages == 0) return W4_ERR_SHAPE;
     static thread_local int attr_dev = -1;
@@ -815,26 +872,26 @@ int launch_ring(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int 
 }
 
 
-template <int M, bool A8>
+template <int M, int AM>
 int dispatch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
              const Act& x, void* y, int out_f32, cudaStream_t st) {
     if ((size_t)N * (size_t)(K / 2) < kRingMaxCodeBytes && plan_for(M, K / 32).stages > 0)
-        return launch_ring<M, A8>(codes, d, m, N, K, x, y, out_f32, st);
-    return dispatch_m<M, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        return launch_ring<M, AM>(codes, d, m, N, K, x, y, out_f32, st);
+    return dispatch_m<M, AM>(codes, d, m, N, K, x, y, out_f32, st);
 }
 
-template <bool A8>
+template <int AM>
 int dispatch_any_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                    const Act& x, int M, void* y, int out_f32, cudaStream_t st) {
     switch (M) {
-        case 1: return dispatch<1, A8>(codes, d, m, N, K, x, y, out_f32, st);
-        case 2: return dispatch<2, A8>(codes, d, m, N, K, x, y, out_f32, st);
-        case 3: return dispatch<3, A8>(codes, d, m, N, K, x, y, out_f32, st);
-        case 4: return dispatch<4, A8>(codes, d, m, N, K, x, y, out_f32, st);
-        case 5: return dispatch<5, A8>(codes, d, m, N, K, x, y, out_f32, st);
-        case 6: return dispatch<6, A8>(codes, d, m, N, K, x, y, out_f32, st);
-        case 7: return dispatch<7, A8>(codes, d, m, N, K, x, y, out_f32, st);
-        default: return dispatch<8, A8>(codes, d, m, N, K, x, y, out_f32, st);
+        case 1: return dispatch<1, AM>(codes, d, m, N, K, x, y, out_f32, st);
+        case 2: return dispatch<2, AM>(codes, d, m, N, K, x, y, out_f32, st);
+        case 3: return dispatch<3, AM>(codes, d, m, N, K, x, y, out_f32, st);
+        case 4: return dispatch<4, AM>(codes, d, m, N, K, x, y, out_f32, st);
+        case 5: return dispatch<5, AM>(codes, d, m, N, K, x, y, out_f32, st);
+        case 6: return dispatch<6, AM>(codes, d, m, N, K, x, y, out_f32, st);
+        case 7: return dispatch<7, AM>(codes, d, m, N, K, x, y, out_f32, st);
+        default: return dispatch<8, AM>(codes, d, m, N, K, x, y, out_f32, st);
     }
 }
 
@@ -862,7 +919,7 @@ extern "C" int w4_gemv(const uint8_t* codes, const uint16_t* d_f16, const uint16
     const int rc = validate(codes, d_f16, m_f16, N, K, x_bf16, x_bf16, x_bf16, M, y, out_dtype);
     if (rc != W4_OK) return rc;
     const Act act{x_bf16, nullptr, nullptr};
-    return dispatch_any_m<false>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
+    return dispatch_any_m<kActBf16>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
                                  out_dtype == W4_OUT_F32, (cudaStream_t)stream);
 }
 
@@ -872,6 +929,16 @@ extern "C" int w4a8_gemv(const uint8_t* codes, const uint16_t* d_f16, const uint
     const int rc = validate(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype);
     if (rc != W4_OK) return rc;
     const Act act{qa, dx, bsum};
-    return dispatch_any_m<true>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
+    return dispatch_any_m<kActInt8>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
                                 out_dtype == W4_OUT_F32, (cudaStream_t)stream);
+}
+
+extern "C" int w4a8_gemv_bf16(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
+                              int64_t N, int64_t K, const uint16_t* x_bf16, int M, void* y,
+                              int out_dtype, void* stream) {
+    const int rc = validate(codes, d_f16, m_f16, N, K, x_bf16, x_bf16, x_bf16, M, y, out_dtype);
+    if (rc != W4_OK) return rc;
+    const Act act{x_bf16, nullptr, nullptr};
+    return dispatch_any_m<kActBf16ToInt8>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
+                                          out_dtype == W4_OUT_F32, (cudaStream_t)stream);
 }

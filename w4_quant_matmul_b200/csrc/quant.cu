@@ -56,12 +56,7 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __rest
             const float rcp = __frcp_rn(scale);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float q0 = f[j] * rcp;
-                const float q = fmaf(fmaf(-q0, scale, f[j]), rcp, q0);
-                float qf = rintf(q);
-                if (fabsf(fabsf(q - qf) - 0.5f) < 0x1p-14f) qf = rintf(__fdiv_rn(f[j], scale));
-                qf = fminf(fmaxf(qf, -127.0f), 127.0f);
-                const int qi = (int)qf;
+                const int qi = w4::q8_code(f[j], scale, rcp);
                 sum += qi;
                 packed[j >> 2] |= ((uint32_t)qi & 0xFFu) << (8 * (j & 3));
             }
