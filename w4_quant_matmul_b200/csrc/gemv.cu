@@ -49,6 +49,11 @@
 //    row kernel is launched in plain stream order (its dependency wait is
 //    then a no-op): measured in a five-GEMV decode step, its CTAs launched
 //    early behind a ring kernel cost more than the overlap gained.
+//  * Activation forms.  The same kernels also take the activations as int8
+//    blocks of 32 (qa, dx, S from q8_quantize_act: the 32-code chunk is one
+//    block, two dp4a per code word give its exact dot product P, then
+//    y += d * (dx * P) + m * (dx * S)), or as bf16 quantised to those blocks in
+//    shared memory with the quantiser's own code function.
 // Integer sums are exact and the float reductions run in a fixed order:
 // results are bitwise deterministic (for a given shape, which fixes the kernel).
 #include <cuda_bf16.h>
