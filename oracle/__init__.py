@@ -1,4 +1,5 @@
-"""CPU oracle for the W4-G256 quantized matmul -- TEST INFRASTRUCTURE ONLY.
+"""CPU oracle for the W4-G256 quantized matmul (and its group-32 variant) --
+TEST INFRASTRUCTURE ONLY.
 
 Thin ctypes wrapper over ``w4_oracle.c`` (plain C, fp64/int64 reductions).
 Only the test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
@@ -57,9 +58,12 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
         "oracle_pack_codes": [P, I, I, P],
         "oracle_unpack": [P, I, I, P],
         "oracle_w4_pack": [P, I, I, P, P, P],
+        "oracle_w4_pack_grouped": [P, I, I, I, P, P, P],
         "oracle_q8_quantize": [P, I, I, P, P, P],
         "oracle_gemv_f64_rows": [P, P, P, I, I, P, I, I, I, P],
         "oracle_gemv_rows": [P, P, P, I, I, P, I, I, I, P],
+        "oracle_gemv_f64_rows_grouped": [P, P, P, I, I, I, P, I, I, I, P],
+        "oracle_gemv_rows_grouped": [P, P, P, I, I, I, P, I, I, I, P],
         "oracle_mmq_blockdots": [P, I, I, P, I, P],
         "oracle_mmq_rows": [P, P, P, I, I, P, P, P, I, I, I, P],
     }
@@ -127,16 +131,21 @@ class Oracle:
         _check(self.lib.oracle_unpack(_ptr(codes), N, K, _ptr(out)), "unpack")
         return out
 
-    def w4_pack(self, w: np.ndarray):
-        """fp32 W[N,K] -> (codes u8[N,K/2], d fp16-bits[N,G], m fp16-bits[N,G])."""
+    def w4_pack(self, w: np.ndarray, group: int = GROUP):
+        """fp32 W[N,K] -> (codes u8[N,K/2], d fp16-bits[N,G], m fp16-bits[N,G]),
+        G = K / group (256: W4-G256; 32: the group-32 scheme)."""
         w = np.ascontiguousarray(w, dtype=np.float32)
         N, K = w.shape
         codes = np.empty((N, K // 2), np.uint8)
-        G = K // GROUP
+        G = K // group
         d = np.empty((N, G), np.uint16)
         m = np.empty((N, G), np.uint16)
-        _check(self.lib.oracle_w4_pack(_ptr(w), N, K, _ptr(codes), _ptr(d), _ptr(m)),
-               "w4_pack")
+        if group == GROUP:
+            rc = self.lib.oracle_w4_pack(_ptr(w), N, K, _ptr(codes), _ptr(d), _ptr(m))
+        else:
+            rc = self.lib.oracle_w4_pack_grouped(_ptr(w), N, K, group, _ptr(codes), _ptr(d),
+                                                 _ptr(m))
+        _check(rc, "w4_pack")
         return codes, d, m
 
     # -- activation quantiser --------------------------------------------
@@ -153,8 +162,9 @@ class Oracle:
         return qa, dx, S
 
     # -- products ----------------------------------------------------------
-    def gemv(self, codes, d, m, x_bf16, rows: tuple[int, int] | None = None) -> np.ndarray:
-        """y[M, rows] in fp64 for bf16-bits x[M,K]."""
+    def gemv(self, codes, d, m, x_bf16, rows: tuple[int, int] | None = None,
+             group: int = GROUP) -> np.ndarray:
+        """y[M, rows] in fp64 for bf16-bits x[M,K]; d, m are [N, K/group]."""
         codes = np.ascontiguousarray(codes, np.uint8)
         d = np.ascontiguousarray(d, np.uint16)
         m = np.ascontiguousarray(m, np.uint16)
@@ -163,11 +173,16 @@ class Oracle:
         M, K = x.shape
         n0, n1 = rows if rows is not None else (0, N)
         y = np.empty((M, n1 - n0), np.float64)
-        _check(self.lib.oracle_gemv_rows(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x), M,
-                                         n0, n1, _ptr(y)), "gemv")
+        if group == GROUP:
+            rc = self.lib.oracle_gemv_rows(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x), M,
+                                           n0, n1, _ptr(y))
+        else:
+            rc = self.lib.oracle_gemv_rows_grouped(_ptr(codes), _ptr(d), _ptr(m), N, K, group,
+                                                   _ptr(x), M, n0, n1, _ptr(y))
+        _check(rc, "gemv")
         return y
 
-    def gemv_f64(self, codes, d, m, x: np.ndarray, rows=None) -> np.ndarray:
+    def gemv_f64(self, codes, d, m, x: np.ndarray, rows=None, group: int = GROUP) -> np.ndarray:
         """Same product with fp64 activations x[M,K]."""
         codes = np.ascontiguousarray(codes, np.uint8)
         d = np.ascontiguousarray(d, np.uint16)
@@ -177,8 +192,13 @@ class Oracle:
         M, K = x.shape
         n0, n1 = rows if rows is not None else (0, N)
         y = np.empty((M, n1 - n0), np.float64)
-        _check(self.lib.oracle_gemv_f64_rows(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x),
-                                             M, n0, n1, _ptr(y)), "gemv_f64")
+        if group == GROUP:
+            rc = self.lib.oracle_gemv_f64_rows(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x),
+                                               M, n0, n1, _ptr(y))
+        else:
+            rc = self.lib.oracle_gemv_f64_rows_grouped(_ptr(codes), _ptr(d), _ptr(m), N, K,
+                                                       group, _ptr(x), M, n0, n1, _ptr(y))
+        _check(rc, "gemv_f64")
         return y
 
     def mmq_blockdots(self, codes, qa) -> np.ndarray:

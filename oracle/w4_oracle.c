@@ -21,7 +21,9 @@
  * the W4-G256 definition: W[N,K], K a multiple of 256, groups of 256 along K,
  * 4-bit codes q in [0,15] with one fp16 scale d and one fp16 min m per group,
  * w = d*q + m; activations for the W4A8 product are int8 per 32-element block
- * with an fp32 scale and an int32 block sum.  Readings where the pages are
+ * with an fp32 scale and an int32 block sum.  The weight quantiser and the
+ * dequantised product also take a group size, for the group-32 variant of the
+ * same format (one d and m per 32 weights).  Readings where the pages are
  * silent (nibble order, rounding rules, scale formula) are listed in the
  * repository's design notes and restated at each function below.
  *
@@ -151,30 +153,47 @@ int oracle_unpack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *q) {
 }
 
 /* ------------------------------------------------------------------------ */
-/* weight quantiser (min/max per group of 256)                              */
+/* weight quantiser (min/max per group)                                     */
 /* ------------------------------------------------------------------------ */
 
-/* w: fp32 [N][K], K % 256 == 0  ->  codes [N][K/2], d, m: fp16 bits [N][K/256].
+/* w: fp32 [N][K]  ->  codes [N][K/2], d, m: fp16 bits [N][K/group], for a
+ * group size `group` that is even and divides K: 256 for W4-G256, 32 for the
+ * asymmetric int4 group-32 W4A16 scheme ("ROCM_OCTAVE", "Validation": its
+ * models are W4A16, int4, group 32; the sparse-attention evaluation's "Setup"
+ * calls the scheme asymmetric, g32), read as the same w = d*q + m form with
+ * one d and one m per 32 weights.
  *
  * Per (row, group), in fp32:
- *   mn, mx = min, max of the 256 weights
+ *   mn, mx = min, max of the group's weights
  *   d16 = fp16(RN((mx - mn) / 15)),  m16 = fp16(RN(mn))
  *   q   = 0 for every weight if d16 == 0, else
  *         clamp(rint((w - float(m16)) / float(d16)), 0, 15)   (ties to even)
  * so that w is approximated by float(d16)*q + float(m16), the dequantisation
  * rule w = d*q + m of the format.  Using the fp16-rounded d and m inside the
  * code computation keeps codes consistent with what is stored. */
-int oracle_w4_pack(const float *w, int64_t N, int64_t K, uint8_t *codes,
-                   uint16_t *d, uint16_t *m) {
-    if (N < 0 || K < 0 || (K % ORACLE_GROUP)) return -1;
-    const int64_t G = K / ORACLE_GROUP;
+static unsigned weight_code(float w, float df, float mf) {
+    if (df == 0.0f) return 0;
+    float num = w - mf;
+#ifdef ORACLE_MUTANT_ROUND_AWAY
+    float qf = roundf(num / df);
+#else
+    float qf = rintf(num / df);
+#endif
+    if (qf < 0.0f) qf = 0.0f;
+    if (qf > 15.0f) qf = 15.0f;
+    return (unsigned)qf;
+}
+
+int oracle_w4_pack_grouped(const float *w, int64_t N, int64_t K, int64_t group,
+                           uint8_t *codes, uint16_t *d, uint16_t *m) {
+    if (N < 0 || K < 0 || group < 2 || (group & 1) || (K % group)) return -1;
+    const int64_t G = K / group;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n) {
-        uint8_t qrow[ORACLE_GROUP];
         for (int64_t g = 0; g < G; ++g) {
-            const float *wg = w + n * K + g * ORACLE_GROUP;
+            const float *wg = w + n * K + g * group;
             float mn = wg[0], mx = wg[0];
-            for (int i = 1; i < ORACLE_GROUP; ++i) {
+            for (int64_t i = 1; i < group; ++i) {
                 if (wg[i] < mn) mn = wg[i];
                 if (wg[i] > mx) mx = wg[i];
             }
@@ -182,28 +201,14 @@ int oracle_w4_pack(const float *w, int64_t N, int64_t K, uint8_t *codes,
             uint16_t d16 = float_to_f16_bits(range / 15.0f);
             uint16_t m16 = float_to_f16_bits(mn);
             float df = f16_bits_to_float(d16), mf = f16_bits_to_float(m16);
-            for (int i = 0; i < ORACLE_GROUP; ++i) {
-                float qf;
-                if (df == 0.0f) {
-                    qf = 0.0f;
-                } else {
-                    float num = wg[i] - mf;
-#ifdef ORACLE_MUTANT_ROUND_AWAY
-                    qf = roundf(num / df);
-#else
-                    qf = rintf(num / df);
-#endif
-                    if (qf < 0.0f) qf = 0.0f;
-                    if (qf > 15.0f) qf = 15.0f;
-                }
-                qrow[i] = (uint8_t)qf;
-            }
-            uint8_t *crow = codes + n * (K / 2) + g * (ORACLE_GROUP / 2);
-            for (int j = 0; j < ORACLE_GROUP / 2; ++j) {
+            uint8_t *crow = codes + n * (K / 2) + g * (group / 2);
+            for (int64_t j = 0; j < group / 2; ++j) {
+                unsigned lo = weight_code(wg[2 * j], df, mf);
+                unsigned hi = weight_code(wg[2 * j + 1], df, mf);
 #ifdef ORACLE_MUTANT_SWAP_NIBBLES
-                crow[j] = (uint8_t)(qrow[2 * j + 1] | (qrow[2 * j] << 4));
+                crow[j] = (uint8_t)(hi | (lo << 4));
 #else
-                crow[j] = (uint8_t)(qrow[2 * j] | (qrow[2 * j + 1] << 4));
+                crow[j] = (uint8_t)(lo | (hi << 4));
 #endif
             }
             d[n * G + g] = d16;
@@ -211,6 +216,12 @@ int oracle_w4_pack(const float *w, int64_t N, int64_t K, uint8_t *codes,
         }
     }
     return 0;
+}
+
+/* The W4-G256 packer: groups of 256. */
+int oracle_w4_pack(const float *w, int64_t N, int64_t K, uint8_t *codes,
+                   uint16_t *d, uint16_t *m) {
+    return oracle_w4_pack_grouped(w, N, K, ORACLE_GROUP, codes, d, m);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -271,17 +282,18 @@ int oracle_q8_quantize(const uint16_t *x, int64_t M, int64_t K, int8_t *qa,
 
 /* The definition written out:
  *   y[t][n] = sum_k ( d[n][g(k)] * q[n][k] + m[n][g(k)] ) * x[t][k],
- * g(k) = k / 256, each weight dequantised on its own, accumulated in fp64 in
- * plain k order.  x is fp64 [M][K]; y is fp64 [M][N].  Rows [n0, n1) only
+ * g(k) = k / group (group = 256 for W4-G256, 32 for the g32 scheme; d and m
+ * are [N][K/group]), each weight dequantised on its own, accumulated in fp64
+ * in plain k order.  x is fp64 [M][K]; y is fp64 [M][N].  Rows [n0, n1) only
  * (the full product is n0 = 0, n1 = N); y holds M x (n1 - n0) values, row
  * stride (n1 - n0). */
-int oracle_gemv_f64_rows(const uint8_t *codes, const uint16_t *d,
-                         const uint16_t *m, int64_t N, int64_t K,
-                         const double *x, int64_t M, int64_t n0, int64_t n1,
-                         double *y) {
-    if (N < 0 || K < 0 || (K % ORACLE_GROUP) || M < 0) return -1;
+int oracle_gemv_f64_rows_grouped(const uint8_t *codes, const uint16_t *d,
+                                 const uint16_t *m, int64_t N, int64_t K,
+                                 int64_t group, const double *x, int64_t M,
+                                 int64_t n0, int64_t n1, double *y) {
+    if (N < 0 || K < 0 || group < 2 || (group & 1) || (K % group) || M < 0) return -1;
     if (n0 < 0 || n1 > N || n0 > n1) return -1;
-    const int64_t G = K / ORACLE_GROUP;
+    const int64_t G = K / group;
     const int64_t W = n1 - n0;
 #pragma omp parallel for schedule(static)
     for (int64_t n = n0; n < n1; ++n) {
@@ -290,10 +302,12 @@ int oracle_gemv_f64_rows(const uint8_t *codes, const uint16_t *d,
             double acc = 0.0;
             for (int64_t k = 0; k < K; ++k) {
 #ifdef ORACLE_MUTANT_GROUP_INDEX
-                int64_t g = (k + ORACLE_BLOCK) / ORACLE_GROUP;
+                int64_t g = (k + ORACLE_BLOCK) / group;
                 if (g >= G) g = G - 1;
-#else
+#elif defined(ORACLE_MUTANT_GROUP_FIXED_256)
                 int64_t g = k / ORACLE_GROUP;
+#else
+                int64_t g = k / group;
 #endif
                 double dd = f16_bits_to_double(d[n * G + g]);
                 double mm = f16_bits_to_double(m[n * G + g]);
@@ -309,6 +323,13 @@ int oracle_gemv_f64_rows(const uint8_t *codes, const uint16_t *d,
     return 0;
 }
 
+int oracle_gemv_f64_rows(const uint8_t *codes, const uint16_t *d,
+                         const uint16_t *m, int64_t N, int64_t K,
+                         const double *x, int64_t M, int64_t n0, int64_t n1,
+                         double *y) {
+    return oracle_gemv_f64_rows_grouped(codes, d, m, N, K, ORACLE_GROUP, x, M, n0, n1, y);
+}
+
 int oracle_gemv_f64(const uint8_t *codes, const uint16_t *d, const uint16_t *m,
                     int64_t N, int64_t K, const double *x, int64_t M,
                     double *y) {
@@ -317,16 +338,22 @@ int oracle_gemv_f64(const uint8_t *codes, const uint16_t *d, const uint16_t *m,
 
 /* Same product with bf16 activations (bf16 bits [M][K]); the bf16 values are
  * widened exactly to fp64 first.  Rows [n0, n1). */
-int oracle_gemv_rows(const uint8_t *codes, const uint16_t *d, const uint16_t *m,
-                     int64_t N, int64_t K, const uint16_t *x_bf16, int64_t M,
-                     int64_t n0, int64_t n1, double *y) {
+int oracle_gemv_rows_grouped(const uint8_t *codes, const uint16_t *d, const uint16_t *m,
+                             int64_t N, int64_t K, int64_t group, const uint16_t *x_bf16,
+                             int64_t M, int64_t n0, int64_t n1, double *y) {
     if (M < 0 || K < 0) return -1;
     double *xd = (double *)malloc(sizeof(double) * (size_t)(M * K + 1));
     if (!xd) return -2;
     for (int64_t i = 0; i < M * K; ++i) xd[i] = bf16_bits_to_double(x_bf16[i]);
-    int rc = oracle_gemv_f64_rows(codes, d, m, N, K, xd, M, n0, n1, y);
+    int rc = oracle_gemv_f64_rows_grouped(codes, d, m, N, K, group, xd, M, n0, n1, y);
     free(xd);
     return rc;
+}
+
+int oracle_gemv_rows(const uint8_t *codes, const uint16_t *d, const uint16_t *m,
+                     int64_t N, int64_t K, const uint16_t *x_bf16, int64_t M,
+                     int64_t n0, int64_t n1, double *y) {
+    return oracle_gemv_rows_grouped(codes, d, m, N, K, ORACLE_GROUP, x_bf16, M, n0, n1, y);
 }
 
 int oracle_gemv(const uint8_t *codes, const uint16_t *d, const uint16_t *m,

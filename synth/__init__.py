@@ -127,11 +127,12 @@ def tiny(seed: int = 0):
     return codes, d, m, x
 
 
-def quantized_weights_direct(N: int, K: int, seed: int):
-    """Directly drawn W4-G256 weights (no quantiser involved): uniform code
-    bytes, d ~ U(0.001, 0.02), m ~ U(-0.1, 0), as fp16 bits."""
+def quantized_weights_direct(N: int, K: int, seed: int, group: int = GROUP):
+    """Directly drawn W4 weights (no quantiser involved): uniform code bytes,
+    d ~ U(0.001, 0.02), m ~ U(-0.1, 0), as fp16 bits, one d and m per `group`
+    weights (256: W4-G256; 32: the group-32 variant)."""
     rng = np.random.default_rng(seed)
     codes = random_code_bytes(N, K, rng)
-    d = uniform_f16_bits((N, K // GROUP), 0.001, 0.02, rng)
-    m = uniform_f16_bits((N, K // GROUP), -0.1, 0.0, rng)
+    d = uniform_f16_bits((N, K // group), 0.001, 0.02, rng)
+    m = uniform_f16_bits((N, K // group), -0.1, 0.0, rng)
     return codes, d, m

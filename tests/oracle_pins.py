@@ -31,15 +31,15 @@ def _bf16(v) -> np.ndarray:
     return synth.f32_to_bf16_bits(np.asarray(v, np.float32))
 
 
-def _dequant_dense(o, codes, d, m, K):
+def _dequant_dense(o, codes, d, m, K, group=GROUP):
     """Dense fp64 W[N,K] from the oracle's own unpack (pinned separately) and
     numpy broadcasting of the per-group d, m."""
     q = o.unpack(codes, K).astype(np.float64)
     dd = synth.f16_bits_to_f32(d).astype(np.float64)
     mm = synth.f16_bits_to_f32(m).astype(np.float64)
     N = q.shape[0]
-    G = K // GROUP
-    W = q.reshape(N, G, GROUP) * dd[:, :, None] + mm[:, :, None]
+    G = K // group
+    W = q.reshape(N, G, group) * dd[:, :, None] + mm[:, :, None]
     return W.reshape(N, K)
 
 
@@ -323,6 +323,105 @@ def pin_mmq_row_window(o):
     full = o.mmq(codes, d, m, qa, dx, S)
     part = o.mmq(codes, d, m, qa, dx, S, rows=(2, 9))
     assert np.array_equal(part, full[:, 2:9])
+
+
+# --------------------------------------------------------------------------
+# group-32 variant (one d and m per 32 weights; "ROCM_OCTAVE", "Validation":
+# W4A16 int4 group 32, asymmetric)
+# --------------------------------------------------------------------------
+
+G32 = 32
+
+
+def pin_g32_wpack_constant_groups(o):
+    # every 32-group constant, a different constant per group: codes 0, d = +0,
+    # m = the constant, group by group (a 256-wide or shifted group fails)
+    N, K = 2, 256
+    vals = (np.arange(N * (K // G32)).reshape(N, K // G32) * 0.125 - 1.0).astype(np.float32)
+    w = np.repeat(vals, G32, axis=1)
+    codes, d, m = o.w4_pack(w, group=G32)
+    assert d.shape == (N, K // G32) and np.all(d == 0) and np.all(codes == 0)
+    assert np.array_equal(synth.f16_bits_to_f32(m), vals)
+
+
+def pin_g32_wpack_grid_idempotent(o):
+    # weights on the grid w = d*q + m of each 32-group (codes 0 and 15 present,
+    # d = k * 2^-10, m = j * 2^-6, exact in fp16 and fp32) re-quantise to
+    # themselves
+    rng = np.random.default_rng(25)
+    N, K = 5, 512
+    G = K // G32
+    dval = (rng.integers(1, 64, size=(N, G)) * 2.0 ** -10).astype(np.float32)
+    mval = (rng.integers(-32, 32, size=(N, G)) * 2.0 ** -6).astype(np.float32)
+    q = synth.random_codes(N, K, rng)
+    q[:, 0::G32] = 0
+    q[:, 7::G32] = 15
+    w = (q.reshape(N, G, G32).astype(np.float32) * dval[:, :, None]
+         + mval[:, :, None]).reshape(N, K).astype(np.float32)
+    codes, d, m = o.w4_pack(w, group=G32)
+    assert np.array_equal(synth.f16_bits_to_f32(d), dval)
+    assert np.array_equal(synth.f16_bits_to_f32(m), mval)
+    assert np.array_equal(o.unpack(codes, K), q)
+
+
+def pin_g32_wpack_error_bound(o):
+    # |w - (d*q + m)| <= d/2 plus the fp16 rounding of d and m, per 32-group;
+    # each group's extreme weights take codes 0 and 15
+    N, K = 12, 512
+    w = synth.dense_weights(N, K, seed=78)
+    codes, d, m = o.w4_pack(w, group=G32)
+    G = K // G32
+    q = o.unpack(codes, K).astype(np.float64).reshape(N, G, G32)
+    dd = synth.f16_bits_to_f32(d).astype(np.float64)
+    mm = synth.f16_bits_to_f32(m).astype(np.float64)
+    wg = w.reshape(N, G, G32).astype(np.float64)
+    deq = q * dd[:, :, None] + mm[:, :, None]
+    mn, mx = wg.min(axis=2), wg.max(axis=2)
+    slack = np.abs(mm - mn) + 15.0 * np.abs(dd - (mx - mn) / 15.0) + 1e-7
+    assert np.all(np.abs(wg - deq) <= dd[:, :, None] / 2 + slack[:, :, None])
+    assert np.all(q.min(axis=2) == 0) and np.all(q.max(axis=2) == 15)
+
+
+def pin_g32_gemv_library_matmul(o):
+    # brute force: numpy fp64 matmul of the dense matrix built by broadcasting
+    # one (d, m) pair over each 32 weights
+    N, K = 33, 320
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=31, group=G32)
+    x = synth.activations(4, K, seed=32)
+    y = o.gemv(codes, d, m, x, group=G32)
+    W = _dequant_dense(o, codes, d, m, K, group=G32)
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ W.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12), float(np.abs(y - ref).max())
+
+
+def pin_g32_gemv_constant_codes(o):
+    # all codes c: y = sum_g (d_g*c + m_g) * sum_{k in 32-group g} x_k
+    rng = np.random.default_rng(33)
+    N, K = 4, 256
+    G = K // G32
+    for c in (0, 9, 15):
+        codes = np.full((N, K // 2), c | (c << 4), np.uint8)
+        d = synth.uniform_f16_bits((N, G), 0.001, 0.02, rng)
+        m = synth.uniform_f16_bits((N, G), -0.1, 0.0, rng)
+        x = synth.normal_bf16_bits((3, K), rng)
+        y = o.gemv(codes, d, m, x, group=G32)
+        xs = synth.bf16_bits_to_f32(x).astype(np.float64).reshape(3, G, G32).sum(axis=2)
+        dd = synth.f16_bits_to_f32(d).astype(np.float64)
+        mm = synth.f16_bits_to_f32(m).astype(np.float64)
+        ref = xs @ (dd * c + mm).T
+        assert np.allclose(y, ref, rtol=1e-12, atol=1e-12), (c, float(np.abs(y - ref).max()))
+
+
+def pin_g32_gemv_reduces_to_g256(o):
+    # W4-G256 planes repeated over the eight 32-groups of each 256-group are
+    # the same matrix: the group-32 product equals the (separately pinned)
+    # W4-G256 product bit for bit, same weights in the same k order
+    N, K = 9, 768
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=34)
+    x = synth.activations(2, K, seed=35)
+    y256 = o.gemv(codes, d, m, x)
+    y32 = o.gemv(codes, np.repeat(d, 8, axis=1), np.repeat(m, 8, axis=1), x, group=G32)
+    assert np.array_equal(y32, y256)
 
 
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

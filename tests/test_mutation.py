@@ -2,8 +2,9 @@
 
 Each variant is the oracle source compiled with one ``-DORACLE_MUTANT_*``
 macro (a swapped nibble order, a dropped min term, ties rounded away from
-zero, an off-by-one block sum, a shifted group index, a dropped block-sum
-term in the W4A8 product).  The mistake lives in the oracle on the CPU; no GPU
+zero, an off-by-one block sum, a shifted group index, a product that indexes
+d and m by 256-wide groups whatever the group size, a dropped block-sum term
+in the W4A8 product).  The mistake lives in the oracle on the CPU; no GPU
 code is involved.  Every variant must fail at least one pin.
 """
 import pytest
@@ -17,6 +18,7 @@ MUTANTS = [
     "ROUND_AWAY",
     "BLOCKSUM_OFF_BY_ONE",
     "GROUP_INDEX",
+    "GROUP_FIXED_256",
     "MMQ_DROP_BLOCKSUM",
 ]
 
@@ -33,3 +35,6 @@ def test_mutant_is_caught(tmp_path, mutant):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, f"no pin caught the planted mistake {mutant}"
+    if mutant == "GROUP_FIXED_256":
+        # the mistake only shows at group 32: the group-32 pins must see it
+        assert any(name.startswith("pin_g32_") for name in failed), failed

@@ -78,6 +78,14 @@ def test_oracle_rejects_bad_shapes(orc):
         orc.w4_pack(np.zeros((2, 300), np.float32))
     with pytest.raises(ValueError):
         orc.q8_quantize(np.zeros((2, 48), np.uint16))
+    # group 32: K must be a multiple of 32; 256-wide and odd groups too
+    with pytest.raises(ValueError):
+        orc.w4_pack(np.zeros((2, 48), np.float32), group=32)
+    with pytest.raises(ValueError):
+        orc.w4_pack(np.zeros((2, 66), np.float32), group=33)
+    codes, d, m = synth.quantized_weights_direct(3, 96, seed=1, group=32)
+    with pytest.raises(ValueError):
+        orc.gemv(codes, d, m, synth.activations(1, 100, seed=2), group=32)
 
 
 def test_threads_do_not_change_results(orc):
