@@ -723,7 +723,10 @@ def run_reference(args):
 
 def run_case(args):
     """One kernel configuration launched `--reps` times on device-resident
-    synthetic inputs (the command the committed ncu summaries capture)."""
+    synthetic inputs (the command the committed ncu summaries capture).  With
+    --time: 3 untimed launches, then each of the --reps launches timed alone
+    with CUDA events after a 256 MB write that flushes L2; prints the median
+    microseconds per launch and, for the GEMVs, algorithmic GB/s."""
     import torch
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -732,26 +735,55 @@ def run_case(args):
     g.manual_seed(17)
     N, K, M = args.N, args.K, args.M
     w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
-    codes, d, m = w4.w4_pack(w)
+    codes, d, m = (w4.w4_pack_g32 if args.case == "gemv_g32" else w4.w4_pack)(w)
     del w
     torch.cuda.synchronize()
     x = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
-    if args.case == "gemv":
+    nbytes = None
+    if args.case in ("gemv", "gemv_g32"):
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        for _ in range(args.reps):
-            w4.w4_gemv(codes, d, m, x, out_dtype=torch.bfloat16, y=y)
+        gemv = w4.w4_gemv_g32 if args.case == "gemv_g32" else w4.w4_gemv
+        nbytes = sum(t.numel() * t.element_size() for t in (codes, d, m, x, y))
+
+        def launch():
+            gemv(codes, d, m, x, out_dtype=torch.bfloat16, y=y)
     elif args.case == "quant":
         qa, dx, S = w4.q8_quantize_act(x)
-        for _ in range(args.reps):
+
+        def launch():
             w4.q8_quantize_act(x, qa, dx, S)
     else:
         qa, dx, S = w4.q8_quantize_act(x)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        for _ in range(args.reps):
+
+        def launch():
             w4.w4a8_mmq(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y)
+    out = {"case": args.case, "N": N, "K": K, "M": M, "reps": args.reps}
+    if args.time:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            launch()
+        events = []
+        for _ in range(args.reps):
+            flush.zero_()
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record()
+            launch()
+            end.record()
+            events.append((start, end))
+        torch.cuda.synchronize()
+        us = sorted(s.elapsed_time(e) * 1e3 for s, e in events)[len(events) // 2]
+        out["us_per_launch"] = round(us, 2)
+        if nbytes is not None:
+            out["bytes"] = nbytes
+            out["GBps"] = round(nbytes / (us * 1e-6) / 1e9, 1)
+    else:
+        for _ in range(args.reps):
+            launch()
     torch.cuda.synchronize()
     w4.w4_check_device_error()
-    print(json.dumps({"case": args.case, "N": N, "K": K, "M": M, "reps": args.reps, "ok": True}))
+    out["ok"] = True
+    print(json.dumps(out))
 
 
 def main(argv=None):
@@ -763,8 +795,10 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="only the timed batch-1 sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["gemv", "mmq", "quant"],
+    ap.add_argument("--case", choices=["gemv", "gemv_g32", "mmq", "quant"],
                     help="launch one kernel configuration --reps times (profiling)")
+    ap.add_argument("--time", action="store_true",
+                    help="with --case: time each launch alone after an L2 flush")
     ap.add_argument("--N", type=int, default=151936)
     ap.add_argument("--K", type=int, default=2560)
     ap.add_argument("--M", type=int, default=1)

@@ -92,6 +92,16 @@ int w4_check_device_error(void);
 int w4_pack(const float *w, int64_t N, int64_t K, uint8_t *codes,
             uint16_t *d_f16, uint16_t *m_f16, void *stream);
 
+/* w4_pack for the group-32 variant of the format: the asymmetric int4,
+ * group-32 scheme of the W4A16 checkpoints on the ROCM_OCTAVE page
+ * ("Validation": W4A16, int4, group 32; the sparse-attention evaluation's
+ * "Setup": asymmetric, g32), read as the same w = d*q + m form with one fp16
+ * d and one fp16 m per 32 weights.  Same quantiser rule per group of 32.
+ * w: fp32 [N][K]; outputs codes [N][K/2] (nibble order as above), d [N][K/32],
+ * m [N][K/32].  N >= 0, K >= 0, K % 32 == 0.  Errors as w4_pack. */
+int w4_pack_g32(const float *w, int64_t N, int64_t K, uint8_t *codes,
+                uint16_t *d_f16, uint16_t *m_f16, void *stream);
+
 /* Pack one-code-per-byte q [N][K] (values 0..15; higher bits are ignored)
  * into codes [N][K/2] with the nibble order above.  K % 2 == 0 and
  * (N*K) % 32 == 0. */
@@ -114,6 +124,17 @@ int w4_gemv(const uint8_t *codes, const uint16_t *d_f16,
             const uint16_t *m_f16, int64_t N, int64_t K,
             const uint16_t *x_bf16, int M, void *y, int out_dtype,
             void *stream);
+
+/* w4_gemv for group-32 weights (the W4A16 g32 scheme of w4_pack_g32):
+ *   y[t][n] = sum_g ( d[n][g] * sum_{k in g} q[n][k] * x[t][k]
+ *                     + m[n][g] * sum_{k in g} x[t][k] ),  groups of 32,
+ * accumulated in fp32.  codes [N][K/2], d and m [N][K/32] from w4_pack_g32;
+ * x: bf16 [M][K]; y: [M][N] of out_dtype.  1 <= M <= 8, N >= 1, K >= 32,
+ * K % 32 == 0.  Same validation and errors as w4_gemv. */
+int w4_gemv_g32(const uint8_t *codes, const uint16_t *d_f16,
+                const uint16_t *m_f16, int64_t N, int64_t K,
+                const uint16_t *x_bf16, int M, void *y, int out_dtype,
+                void *stream);
 
 /* Decode GEMV on int8 activation blocks ("keep-quant" decode: the
  * activations stay in the Q8_1-style blocks that q8_quantize_act produces, so

@@ -28,7 +28,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for expected in ["w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "w4a8_gemv",
+    for expected in ["w4_pack", "w4_pack_g32", "w4_pack_codes", "w4_unpack", "w4_gemv",
+                     "w4_gemv_g32", "w4a8_gemv",
                      "w4a8_gemv_bf16", "q8_quantize_act",
                      "w4a8_mmq", "w4a8_mmq_workspace_size", "w4_status_string",
                      "w4_abi_version", "w4_last_cuda_error", "w4_check_device_error"]:
@@ -84,6 +85,24 @@ def test_w4a8_gemv_validation(lib):
     assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, FAKE, None, 1, FAKE, 0, None) == L.W4_ERR_NULL
     assert f(FAKE, FAKE, FAKE, 256, 512, MIS, FAKE, FAKE, 1, FAKE, 0, None) == L.W4_ERR_ALIGN
     assert f(FAKE, FAKE, FAKE, 256, 512, FAKE, MIS, FAKE, 1, FAKE, 0, None) == L.W4_ERR_ALIGN
+
+
+def test_g32_validation(lib):
+    from w4_quant_matmul_b200 import _lib as L
+    f = lib.w4_gemv_g32
+    assert f(FAKE, FAKE, FAKE, 256, 48, FAKE, 1, FAKE, 0, None) == L.W4_ERR_SHAPE   # K % 32
+    assert f(FAKE, FAKE, FAKE, 256, 0, FAKE, 1, FAKE, 0, None) == L.W4_ERR_SHAPE    # K < 32
+    assert f(FAKE, FAKE, FAKE, 256, 96, FAKE, 9, FAKE, 0, None) == L.W4_ERR_SHAPE   # M
+    assert f(FAKE, FAKE, FAKE, 256, 96, FAKE, 1, FAKE, 5, None) == L.W4_ERR_SHAPE   # out dtype
+    assert f(None, FAKE, FAKE, 256, 96, FAKE, 1, FAKE, 0, None) == L.W4_ERR_NULL
+    assert f(FAKE, FAKE, MIS, 256, 96, FAKE, 1, FAKE, 0, None) == L.W4_ERR_ALIGN
+    assert lib.w4_pack_g32(FAKE, 4, 48, FAKE, FAKE, FAKE, None) == L.W4_ERR_SHAPE
+    assert lib.w4_pack_g32(None, 4, 96, FAKE, FAKE, FAKE, None) == L.W4_ERR_NULL
+    assert lib.w4_pack_g32(FAKE, 4, 96, MIS, FAKE, FAKE, None) == L.W4_ERR_ALIGN
+    assert lib.w4_pack_g32(FAKE, 0, 96, FAKE, FAKE, FAKE, None) == L.W4_OK   # nothing to do
+    # 256-group rules still hold for the W4-G256 entry points
+    assert lib.w4_gemv(FAKE, FAKE, FAKE, 256, 96, FAKE, 1, FAKE, 0, None) == L.W4_ERR_SHAPE
+    assert lib.w4_pack(FAKE, 4, 96, FAKE, FAKE, FAKE, None) == L.W4_ERR_SHAPE
 
 
 def test_pack_and_quantizer_validation(lib):

@@ -100,6 +100,21 @@ def test_int8_activation_calls(fn):
                    out_dtype=torch.float32)
 
 
+def test_group32_planes():
+    x = _x()
+    codes = torch.zeros((N, K // 2), dtype=torch.uint8)
+    d32 = torch.zeros((N, K // 32), dtype=torch.float16)
+    _reaches_device_check(w4.w4_gemv_g32, codes, d32, d32, x)
+    d256 = torch.zeros((N, K // 256), dtype=torch.float16)
+    _rejects_shape("d", w4.w4_gemv_g32, codes, d256, d32, x)
+    _rejects_shape("m", w4.w4_gemv_g32, codes, d32, d256, x)
+    # and the W4-G256 GEMV refuses group-32 planes
+    _rejects_shape("d", w4.w4_gemv, codes, d32, d32, x)
+    w = torch.zeros((N, K), dtype=torch.float32)
+    _reaches_device_check(w4.w4_pack_g32, w)
+    _rejects_shape("d", w4.w4_pack_g32, w, d=d256)
+
+
 def test_mmq_workspace_is_checked():
     with pytest.raises(TypeError, match="^workspace must be torch.uint8"):
         w4.w4a8_mmq(*_w4a8_args(), workspace=torch.zeros(16, dtype=torch.int32))

@@ -8,9 +8,11 @@ current stream.  There is no CPU path: without the built library, calls raise
 
 Entry points (same names as the C ABI):
     w4_pack(w)                              -> codes, d, m
+    w4_pack_g32(w)                          -> codes, d, m   (groups of 32)
     w4_pack_codes(q)                        -> codes
     w4_unpack(codes, K)                     -> q
     w4_gemv(codes, d, m, x, out_dtype)      -> y
+    w4_gemv_g32(codes, d, m, x, out_dtype)  -> y   (group-32 weights)
     w4a8_gemv(codes, d, m, qa, dx, bsum, out_dtype) -> y   (int8 activations, M <= 8)
     w4a8_gemv_bf16(codes, d, m, x, out_dtype) -> y   (x quantised inside, M <= 8)
     q8_quantize_act(x)                      -> qa, dx, bsum
@@ -24,7 +26,8 @@ from __future__ import annotations
 from ._lib import (LibraryMissing, W4_OK, W4_OUT_BF16, W4_OUT_F32, load, status_string)
 
 __all__ = [
-    "W4Error", "LibraryMissing", "w4_pack", "w4_pack_codes", "w4_unpack", "w4_gemv", "w4a8_gemv",
+    "W4Error", "LibraryMissing", "w4_pack", "w4_pack_g32", "w4_pack_codes", "w4_unpack",
+    "w4_gemv", "w4_gemv_g32", "w4a8_gemv",
     "w4a8_gemv_bf16",
     "q8_quantize_act", "w4a8_mmq", "w4a8_mmq_static", "w4a8_mmq_workspace_size",
     "w4_check_device_error",
@@ -32,6 +35,7 @@ __all__ = [
 ]
 
 GROUP = 256
+GROUP32 = 32
 BLOCK = 32
 
 
@@ -122,9 +126,7 @@ def w4_check_device_error() -> None:
     _check(load().w4_check_device_error(), "w4_check_device_error")
 
 
-def w4_pack(w, codes=None, d=None, m=None, stream=None):
-    """Quantise fp32 W[N,K] (K % 256 == 0) to W4-G256 planes.
-    Returns (codes uint8[N,K/2], d fp16[N,K/256], m fp16[N,K/256])."""
+def _pack(fn: str, group: int, w, codes, d, m, stream):
     torch = _torch()
     _need(w, torch.float32, "w", (None, None))
     N, K = w.shape
@@ -132,15 +134,27 @@ def w4_pack(w, codes=None, d=None, m=None, stream=None):
         codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
     _need(codes, torch.uint8, "codes", (N, _div(K, 2)))
     if d is None:
-        d = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
-    _need(d, torch.float16, "d", (N, _div(K, GROUP)))
+        d = torch.empty((N, K // group), dtype=torch.float16, device=w.device)
+    _need(d, torch.float16, "d", (N, _div(K, group)))
     if m is None:
-        m = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
-    _need(m, torch.float16, "m", (N, _div(K, GROUP)))
+        m = torch.empty((N, K // group), dtype=torch.float16, device=w.device)
+    _need(m, torch.float16, "m", (N, _div(K, group)))
     _on_device(w=w, codes=codes, d=d, m=m)
-    _check(load().w4_pack(_ptr(w), N, K, _ptr(codes), _ptr(d), _ptr(m), _stream(stream)),
-           "w4_pack")
+    _check(getattr(load(), fn)(_ptr(w), N, K, _ptr(codes), _ptr(d), _ptr(m), _stream(stream)),
+           fn)
     return codes, d, m
+
+
+def w4_pack(w, codes=None, d=None, m=None, stream=None):
+    """Quantise fp32 W[N,K] (K % 256 == 0) to W4-G256 planes.
+    Returns (codes uint8[N,K/2], d fp16[N,K/256], m fp16[N,K/256])."""
+    return _pack("w4_pack", GROUP, w, codes, d, m, stream)
+
+
+def w4_pack_g32(w, codes=None, d=None, m=None, stream=None):
+    """Quantise fp32 W[N,K] (K % 32 == 0) to group-32 planes (one d, m per
+    32 weights).  Returns (codes uint8[N,K/2], d fp16[N,K/32], m fp16[N,K/32])."""
+    return _pack("w4_pack_g32", GROUP32, w, codes, d, m, stream)
 
 
 def w4_pack_codes(q, codes=None, stream=None):
@@ -193,13 +207,14 @@ def _output(y, M: int, N: int, oc: int, like):
     return y
 
 
-def _weights(codes, d, m, K: int) -> int:
-    """Check the W4-G256 planes for reduction length K; returns N."""
+def _weights(codes, d, m, K: int, group: int = GROUP) -> int:
+    """Check the weight planes (d, m per `group` weights) for reduction
+    length K; returns N."""
     torch = _torch()
     _need(codes, torch.uint8, "codes", (None, _div(K, 2)))
     N = codes.shape[0]
-    _need(d, torch.float16, "d", (N, _div(K, GROUP)))
-    _need(m, torch.float16, "m", (N, _div(K, GROUP)))
+    _need(d, torch.float16, "d", (N, _div(K, group)))
+    _need(m, torch.float16, "m", (N, _div(K, group)))
     return N
 
 
@@ -226,6 +241,21 @@ def w4_gemv(codes, d, m, x, out_dtype=None, y=None, stream=None):
     _on_device(codes=codes, d=d, m=m, x=x, y=y)
     _check(load().w4_gemv(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x), M, _ptr(y), oc,
                           _stream(stream)), "w4_gemv")
+    return y
+
+
+def w4_gemv_g32(codes, d, m, x, out_dtype=None, y=None, stream=None):
+    """w4_gemv for group-32 weights (w4_pack_g32 planes: d, m fp16[N,K/32]);
+    y[M,N] = x[M,K] @ dequant(W)^T for 1 <= M <= 8, K % 32 == 0."""
+    torch = _torch()
+    _need(x, torch.bfloat16, "x", (None, None))
+    M, K = x.shape
+    N = _weights(codes, d, m, K, GROUP32)
+    oc = _out_code(out_dtype, y)
+    y = _output(y, M, N, oc, x)
+    _on_device(codes=codes, d=d, m=m, x=x, y=y)
+    _check(load().w4_gemv_g32(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(x), M, _ptr(y), oc,
+                              _stream(stream)), "w4_gemv_g32")
     return y
 
 

@@ -33,9 +33,11 @@ SIGNATURES = {
     "w4_last_cuda_error": ([], _INT),
     "w4_check_device_error": ([], _INT),
     "w4_pack": ([_P, _I64, _I64, _P, _P, _P, _P], _INT),
+    "w4_pack_g32": ([_P, _I64, _I64, _P, _P, _P, _P], _INT),
     "w4_pack_codes": ([_P, _I64, _I64, _P, _P], _INT),
     "w4_unpack": ([_P, _I64, _I64, _P, _P], _INT),
     "w4_gemv": ([_P, _P, _P, _I64, _I64, _P, _INT, _P, _INT, _P], _INT),
+    "w4_gemv_g32": ([_P, _P, _P, _I64, _I64, _P, _INT, _P, _INT, _P], _INT),
     "w4a8_gemv": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _INT, _P, _INT, _P], _INT),
     "w4a8_gemv_bf16": ([_P, _P, _P, _I64, _I64, _P, _INT, _P, _INT, _P], _INT),
     "q8_quantize_act": ([_P, _I64, _I64, _P, _P, _P, _P], _INT),

@@ -102,13 +102,18 @@ __device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Group size as a shift of the 32-code chunk index: a chunk c takes the d, m
+// of group c >> GSH (kG256 = 3: groups of 256; kG32 = 0: groups of 32).
+constexpr int kG256 = 3;
+constexpr int kG32 = 0;
+
 template <int RH, int U>
 struct Batch {
     uint4 wq[U][RH];
     uint32_t dm[U][RH];
 };
 
-template <int RH, int U>
+template <int RH, int U, int GSH>
 __device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __restrict__ codes,
                                            const __half* __restrict__ d,
                                            const __half* __restrict__ m, const int (&rows)[RH],
@@ -117,7 +122,7 @@ __device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __res
     for (int u = 0; u < U; ++u) {
         const int c = c0 + 16 * u;
         const bool live = c < c_end;
-        const int g = (live ? c : 0) >> 3;
+        const int g = (live ? c : 0) >> GSH;
 #pragma unroll
         for (int i = 0; i < RH; ++i) {
             if (live) {
@@ -320,13 +325,13 @@ struct MinCtas {
     static constexpr int value = M == 1 ? 3 : (M <= 4 ? 2 : 1);
 };
 
-template <int M, int RH, int U, int AM>
+template <int M, int RH, int U, int AM, int GSH = kG256>
 __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
     int N, int K, int KS, const Act act, void* __restrict__ y, int out_f32) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int C = K >> 5;  // 32-code chunks per row
-    const int G = K >> 8;  // groups per row
+    const int G = K >> (5 + GSH);  // groups per row
     uint4* xq = reinterpret_cast<uint4*>(smem);                                // [M][4][C]
     float* sx = reinterpret_cast<float*>(smem + (size_t)M * 4 * C * 16);         // [M][C]
     float* inv = sx + (size_t)M * C;                                             // [M][C]
@@ -388,7 +393,8 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
     __syncthreads();
     pdl_launch_dependents();
     Batch<RH, U> bt;
-    if (blk < nblocks && active) load_batch(bt, codes, d, m, rows, row_bytes, G, cs + j, ce);
+    if (blk < nblocks && active)
+        load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, cs + j, ce);
 
     for (; blk < nblocks; blk += gridDim.x) {
         float yacc[M][RH];
@@ -398,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
             for (int i = 0; i < RH; ++i) yacc[t][i] = 0.0f;
         if (active) {
             for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
-                if (c0 != cs + j) load_batch(bt, codes, d, m, rows, row_bytes, G, c0, ce);
+                if (c0 != cs + j)
+                    load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, c0, ce);
                 consume_batch<M, RH, U, AM>(bt, xq, sx, inv, C, c0, ce, yacc);
             }
         }
@@ -423,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
             nrows[i] = n < N ? n : N - 1;
         }
         if (nblk < nblocks && active)
-            load_batch(bt, codes, d, m, nrows, row_bytes, G, cs + j, ce);
+            load_batch<RH, U, GSH>(bt, codes, d, m, nrows, row_bytes, G, cs + j, ce);
 
         if (KS == 1) {
 #pragma unroll
@@ -476,11 +483,11 @@ size_t smem_bytes(int M, int C, int KS, int RH) {
            (KS > 1 ? (size_t)KS * rows_per_cta * M * 4 : 0);
 }
 
-template <int M, int RH, int AM>
+template <int M, int RH, int AM, int GSH = kG256>
 int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K, int KS,
            const Act& x, void* y, int out_f32, cudaStream_t st) {
     constexpr int U = 8 / RH;
-    auto kern = w4_gemv_rows_kernel<M, RH, U, AM>;
+    auto kern = w4_gemv_rows_kernel<M, RH, U, AM, GSH>;
     const int C = K / 32;
     const size_t smem = smem_bytes(M, C, KS, RH);
     // Per-instantiation cache: one device, a few shared-memory sizes.
@@ -545,7 +552,7 @@ void pick_split(int N, int C, int sms, int* rh, int* ks) {
     *ks = k;
 }
 
-template <int M, int AM>
+template <int M, int AM, int GSH = kG256>
 int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                const Act& x, void* y, int out_f32, cudaStream_t st) {
     int rh, ks;
@@ -553,10 +560,11 @@ int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N
     if (M >= 4 && rh > 2) rh = 2;  // register budget: M * RH accumulators twice
     if (smem_bytes(M, K / 32, ks, rh) > (size_t)kSmemBudget) ks = 1;
     if constexpr (M < 4) {
-        if (rh == 4) return launch_rows<M, 4, AM>(codes, d, m, N, K, ks, x, y, out_f32, st);
+        if (rh == 4)
+            return launch_rows<M, 4, AM, GSH>(codes, d, m, N, K, ks, x, y, out_f32, st);
     }
-    if (rh >= 2) return launch_rows<M, 2, AM>(codes, d, m, N, K, ks, x, y, out_f32, st);
-    return launch_rows<M, 1, AM>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    if (rh >= 2) return launch_rows<M, 2, AM, GSH>(codes, d, m, N, K, ks, x, y, out_f32, st);
+    return launch_rows<M, 1, AM, GSH>(codes, d, m, N, K, ks, x, y, out_f32, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -900,11 +908,28 @@ int dispatch_any_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, i
     }
 }
 
-// Host validation shared by both entry points; W4_OK if the call may launch.
+// Group-32 weights: the row kernel at every stream size (the ring kernel
+// stages d, m per 256-group).
+int dispatch_g32(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
+                 const Act& x, int M, void* y, int out_f32, cudaStream_t st) {
+    switch (M) {
+        case 1: return dispatch_m<1, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+        case 2: return dispatch_m<2, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+        case 3: return dispatch_m<3, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+        case 4: return dispatch_m<4, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+        case 5: return dispatch_m<5, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+        case 6: return dispatch_m<6, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+        case 7: return dispatch_m<7, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+        default: return dispatch_m<8, kActBf16, kG32>(codes, d, m, N, K, x, y, out_f32, st);
+    }
+}
+
+// Host validation shared by the entry points; W4_OK if the call may launch.
+// K must be a multiple of the group size (256, or 32 for group-32 weights).
 int validate(const void* codes, const void* d, const void* m, int64_t N, int64_t K,
              const void* a0, const void* a1, const void* a2, int M, const void* y,
-             int out_dtype) {
-    if (M < 1 || M > 8 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
+             int out_dtype, int group = 256) {
+    if (M < 1 || M > 8 || N < 1 || K < group || K % group != 0) return W4_ERR_SHAPE;
     if (N > (int64_t)1 << 30 || K > (int64_t)1 << 20) return W4_ERR_SHAPE;
     if (out_dtype != W4_OUT_BF16 && out_dtype != W4_OUT_F32) return W4_ERR_SHAPE;
     if (!codes || !d || !m || !a0 || !a1 || !a2 || !y) return W4_ERR_NULL;
@@ -946,4 +971,15 @@ extern "C" int w4a8_gemv_bf16(const uint8_t* codes, const uint16_t* d_f16, const
     const Act act{x_bf16, nullptr, nullptr};
     return dispatch_any_m<kActBf16ToInt8>(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
                                           out_dtype == W4_OUT_F32, (cudaStream_t)stream);
+}
+
+extern "C" int w4_gemv_g32(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
+                           int64_t N, int64_t K, const uint16_t* x_bf16, int M, void* y,
+                           int out_dtype, void* stream) {
+    const int rc =
+        validate(codes, d_f16, m_f16, N, K, x_bf16, x_bf16, x_bf16, M, y, out_dtype, 32);
+    if (rc != W4_OK) return rc;
+    const Act act{x_bf16, nullptr, nullptr};
+    return dispatch_g32(codes, d_f16, m_f16, (int)N, (int)K, act, M, y,
+                        out_dtype == W4_OUT_F32, (cudaStream_t)stream);
 }

@@ -12,34 +12,49 @@
 namespace {
 
 constexpr int kGroup = 256;
+constexpr int kGroup32 = 32;
 
-// One warp per (row, group): each lane owns 8 consecutive weights.
+// One pass of a warp covers 32 / (GROUP / 8) consecutive (row, group) units:
+// GROUP / 8 lanes per group, each owning 8 consecutive weights (one warp per
+// group at 256, eight groups per warp at 32).
 //   mn, mx -> d16 = fp16_rn((mx - mn) / 15), m16 = fp16_rn(mn)
 //   q = d16 == 0 ? 0 : clamp(rint((w - m16) / d16), 0, 15)
 // All fp32 operations are the IEEE round-to-nearest intrinsics so that the
 // result does not depend on contraction or fast-math settings.
+template <int GROUP>
 __global__ void __launch_bounds__(256) w4_pack_kernel(const float* __restrict__ w, int64_t N,
                                                       int64_t K, uint8_t* __restrict__ codes,
                                                       __half* __restrict__ d,
                                                       __half* __restrict__ m) {
-    const int64_t G = K / kGroup;
+    constexpr int kLanes = GROUP / 8;       // lanes per group
+    constexpr int kPerPass = 32 / kLanes;   // groups per warp pass
+    static_assert(kLanes >= 1 && kLanes <= 32 && 32 % kLanes == 0, "group of 8..256");
+    const int64_t G = K / GROUP;
     const int64_t groups = N * G;
     const int lane = threadIdx.x & 31;
+    const int sub = lane / kLanes, part = lane % kLanes;
     const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t gi = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); gi < groups;
-         gi += warps_total) {
-        const int64_t n = gi / G, g = gi % G;
-        const float4* src = reinterpret_cast<const float4*>(w + n * K + g * kGroup + lane * 8);
-        float4 a = __ldg(src), b = __ldg(src + 1);
-        float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    for (int64_t base = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kPerPass;
+         base < groups; base += warps_total * kPerPass) {
+        const int64_t gi = base + sub;
+        const bool live = gi < groups;  // the same for all lanes of a group
+        const int64_t n = live ? gi / G : 0, g = live ? gi % G : 0;
+        float v[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+        if (live) {
+            const float4* src = reinterpret_cast<const float4*>(w + n * K + g * GROUP + part * 8);
+            const float4 a = __ldg(src), b = __ldg(src + 1);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
         float mn = v[0], mx = v[0];
 #pragma unroll
         for (int i = 1; i < 8; ++i) {
             mn = fminf(mn, v[i]);
             mx = fmaxf(mx, v[i]);
         }
+        // xor offsets below kLanes stay inside the group's lanes
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
+        for (int off = kLanes / 2; off > 0; off >>= 1) {
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         }
@@ -57,10 +72,12 @@ __global__ void __launch_bounds__(256) w4_pack_kernel(const float* __restrict__ 
             }
             packed |= (uint32_t)qf << (4 * i);
         }
-        reinterpret_cast<uint32_t*>(codes + n * (K / 2) + g * (kGroup / 2))[lane] = packed;
-        if (lane == 0) {
-            d[n * G + g] = d16;
-            m[n * G + g] = m16;
+        if (live) {
+            reinterpret_cast<uint32_t*>(codes + n * (K / 2) + g * (GROUP / 2))[part] = packed;
+            if (part == 0) {
+                d[n * G + g] = d16;
+                m[n * G + g] = m16;
+            }
         }
     }
 }
@@ -133,13 +150,10 @@ int grid_for(int64_t work, int threads) {
     return (int)blocks;
 }
 
-}  // namespace
-
-extern "C" {
-
-int w4_pack(const float* w, int64_t N, int64_t K, uint8_t* codes, uint16_t* d_f16,
-            uint16_t* m_f16, void* stream) {
-    if (N < 0 || K < 0 || K % kGroup != 0) return W4_ERR_SHAPE;
+template <int GROUP>
+int pack_grouped(const float* w, int64_t N, int64_t K, uint8_t* codes, uint16_t* d_f16,
+                 uint16_t* m_f16, void* stream) {
+    if (N < 0 || K < 0 || K % GROUP != 0) return W4_ERR_SHAPE;
     if (N == 0 || K == 0) return W4_OK;
     if (!w || !codes || !d_f16 || !m_f16) return W4_ERR_NULL;
     if (!w4::aligned16(w) || !w4::aligned16(codes) || !w4::aligned16(d_f16) ||
@@ -147,10 +161,25 @@ int w4_pack(const float* w, int64_t N, int64_t K, uint8_t* codes, uint16_t* d_f1
         return W4_ERR_ALIGN;
     int rc = w4::check_device();
     if (rc != W4_OK) return rc;
-    const int64_t groups = N * (K / kGroup);
-    w4_pack_kernel<<<grid_for(groups * 32, 256), 256, 0, (cudaStream_t)stream>>>(
+    // one thread per 8 weights: N * K / 8 threads in warp passes
+    const int64_t threads = N * (K / 8);
+    w4_pack_kernel<GROUP><<<grid_for(threads, 256), 256, 0, (cudaStream_t)stream>>>(
         w, N, K, codes, reinterpret_cast<__half*>(d_f16), reinterpret_cast<__half*>(m_f16));
     return w4::launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int w4_pack(const float* w, int64_t N, int64_t K, uint8_t* codes, uint16_t* d_f16,
+            uint16_t* m_f16, void* stream) {
+    return pack_grouped<kGroup>(w, N, K, codes, d_f16, m_f16, stream);
+}
+
+int w4_pack_g32(const float* w, int64_t N, int64_t K, uint8_t* codes, uint16_t* d_f16,
+                uint16_t* m_f16, void* stream) {
+    return pack_grouped<kGroup32>(w, N, K, codes, d_f16, m_f16, stream);
 }
 
 int w4_pack_codes(const uint8_t* q, int64_t N, int64_t K, uint8_t* codes, void* stream) {
