@@ -54,6 +54,10 @@
 //    block, two dp4a per code word give its exact dot product P, then
 //    y += d * (dx * P) + m * (dx * S)), or as bf16 quantised to those blocks in
 //    shared memory with the quantiser's own code function.
+//  * Group size.  The row kernel applies d and m per 32-code chunk, taking
+//    those of group c >> GSH: GSH = 3 for W4-G256, 0 for group-32 weights
+//    (the asymmetric int4 group-32 scheme of the ROCM_OCTAVE page,
+//    "Validation"), which always take the row kernel.
 // Integer sums are exact and the float reductions run in a fixed order:
 // results are bitwise deterministic (for a given shape, which fixes the kernel).
 #include <cuda_bf16.h>

@@ -3,8 +3,11 @@
 // Format: groups of 256 consecutive k per row, 4-bit codes plus one fp16
 // scale d and one fp16 min m per group, w = d*q + m ("HFQ4-G256", hipfire
 // MMQ prefill article).  Byte j of a code row holds k = 2j in bits 0-3 and
-// k = 2j+1 in bits 4-7.  These kernels are off the timed path (weights are
-// packed once); they are written for exactness first, bandwidth second.
+// k = 2j+1 in bits 4-7.  The same quantiser also packs groups of 32 (the
+// asymmetric int4 group-32 W4A16 scheme of the ROCM_OCTAVE page,
+// "Validation"), with d and m planes of K/32 columns.  These kernels are off
+// the timed path (weights are packed once); they are written for exactness
+// first, bandwidth second.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
