@@ -18,7 +18,9 @@ shapes, TOPS), the activation quantiser (GB/s) and the graph-captured
 per-token chain (36 layers x 4 shapes + lm_head, tok/s-equivalent).
 
 One JSON line is printed by rank 0.  `--impl reference` times the CPU oracle
-on a bounded sample of the same workload instead.
+on a bounded sample of the same workload instead.  `--case gemv|gemv_g32|mmq|
+quant` launches one kernel configuration `--reps` times (the commands the
+committed ncu summaries capture); with `--time` each launch is timed alone.
 """
 from __future__ import annotations
 

@@ -10,6 +10,8 @@
  *                            k = 2j+1 in bits 4-7
  *     d      fp16  [N][K/256] (raw IEEE binary16 bits)
  *     m      fp16  [N][K/256]
+ *   Group-32 weights (w4_pack_g32, w4_gemv_g32) use the same codes plane with
+ *   d and m planes of [N][K/32], one pair per 32 consecutive k; K % 32 == 0.
  *   Activations are bf16 [M][K] row-major (raw bits).  For the W4A8 product
  *   they are first quantised per 32-element block (the Q8_1-style MMQ layout
  *   the article pre-quantises prefill activations to):
