@@ -63,6 +63,26 @@ def test_worked_examples(orc):
     assert y.tolist() == e["y"]
 
 
+def test_worked_examples_group32(orc):
+    ex = {e["name"]: e for e in json.load(open(GOLDEN))["g32"]}
+
+    e = ex["pack_two_ramps"]
+    k = np.arange(64)
+    w = np.where(k < 32, (k % 16) / 16.0, -0.5 + (k % 16) / 8.0).astype(np.float32)[None, :]
+    codes, d, m = orc.w4_pack(w, group=e["group"])
+    assert synth.f16_bits_to_f32(d).tolist() == e["d"]
+    assert synth.f16_bits_to_f32(m).tolist() == e["m"]
+    assert orc.unpack(codes, 64)[0].tolist() == (k % 16).tolist()
+
+    e = ex["gemv_two_groups"]
+    q = np.where(k < 32, k % 16, 15 - k % 16)[None, :]
+    x = np.ones((2, 64))
+    x[1, 32:] = -1
+    y = orc.gemv(_codes_from_rule(orc, q), _f16(e["d"]), _f16(e["m"]), _bf16(x),
+                 group=e["group"])
+    assert y.tolist() == e["y"]
+
+
 def test_tiny_case_runs_fast(orc):
     codes, d, m, x = synth.tiny(0)
     t0 = time.perf_counter()
