@@ -103,17 +103,21 @@ def source_hash(*files: str) -> str:
 
 
 def load_traffic(kernel_file: str, key: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    """(DRAM bytes per launch, source): the bytes from a committed ncu summary
+    if it was taken on the current kernel source, else None and the reason."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
-        return None
+        return None, "no profiles/traffic.json"
     with open(path) as f:
         t = json.load(f)
     e = t.get(key)
-    if not e or e.get("source_hash") != source_hash(kernel_file):
-        return None
-    return e.get("dram_bytes_per_launch")
+    if not e:
+        return None, f"no entry {key} in profiles/traffic.json"
+    current = source_hash(kernel_file)
+    if e.get("source_hash") != current:
+        return None, (f"ncu counters ({e.get('capture')}) were taken on {kernel_file} "
+                      f"{e.get('source_hash')}; the source is now {current}")
+    return e.get("dram_bytes_per_launch"), f"ncu capture {e.get('capture')}"
 
 
 class ClockSampler:
@@ -556,10 +560,12 @@ def run_ours(args):
     dom_s = dom_ms / 1e3
     achieved = dom_bytes / dom_s / 1e9
     isolated = dom_bytes / (per_shape_ms[4] / 1e3) / 1e9
-    traffic = load_traffic("w4_quant_matmul_b200/csrc/gemv.cu", "w4_gemv_lm_head_m1")
+    traffic, traffic_source = load_traffic("w4_quant_matmul_b200/csrc/gemv.cu",
+                                           "w4_gemv_lm_head_m1")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic, "kernel": "w4_gemv_rows_kernel (151936x2560, M=1)",
+                "traffic": traffic, "traffic_source": traffic_source,
+                "kernel": "w4_gemv_rows_kernel (151936x2560, M=1)",
                 "duration_us": round(dom_ms * 1e3, 2),
                 "timing": "8 back-to-back launches per CUDA graph, alternating 200 MB weight copies",
                 "isolated_achieved": round(isolated, 1),

@@ -52,3 +52,25 @@ def test_algorithmic_bytes():
     # the five decode shapes stream 253 MB per step, 2.078 GB per chain token
     step = sum(bench.gemv_bytes(n, k, 1) for n, k in bench.SHAPES)
     assert 250e6 < step < 256e6
+
+
+def test_traffic_is_used_only_for_the_source_it_was_taken_on(tmp_path, monkeypatch):
+    import bench
+    kernel = "w4_quant_matmul_b200/csrc/gemv.cu"
+    (tmp_path / "profiles").mkdir()
+    entry = {"dram_bytes_per_launch": 123, "capture": "profiles/x.md"}
+
+    def write(h):
+        with open(tmp_path / "profiles" / "traffic.json", "w") as f:
+            json.dump({"k": dict(entry, source_hash=h)}, f)
+
+    # the hash is read from the real kernel source; the table from tmp_path
+    current = bench.source_hash(kernel)
+    monkeypatch.setattr(bench, "source_hash", lambda f: current if f == kernel else "")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    write(current)
+    assert bench.load_traffic(kernel, "k") == (123, "ncu capture profiles/x.md")
+    write("0" * 16)
+    value, why = bench.load_traffic(kernel, "k")
+    assert value is None and current in why and "0" * 16 in why
+    assert bench.load_traffic(kernel, "other")[0] is None
