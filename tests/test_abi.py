@@ -154,3 +154,33 @@ def test_product_package_does_not_import_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, fn)).read()
                 assert "oracle" not in src.lower(), fn
+
+
+def test_without_a_device_valid_calls_fail_loudly(lib):
+    # no CPU path: with valid arguments and no usable CUDA device, every entry
+    # point stops at the device check and returns an error (nothing computed)
+    import torch
+    from w4_quant_matmul_b200 import _lib as L
+    if torch.cuda.is_available() or lib.w4_check_device_error() == L.W4_OK:
+        pytest.skip("a CUDA device is present; this checks the no-device branch only")
+    M, N, K = 128, 256, 512
+    ws = lib.w4a8_mmq_workspace_size(M, N, K)
+    calls = {
+        "w4_pack": lambda: lib.w4_pack(FAKE, N, K, FAKE, FAKE, FAKE, None),
+        "w4_pack_g32": lambda: lib.w4_pack_g32(FAKE, N, K, FAKE, FAKE, FAKE, None),
+        "w4_pack_codes": lambda: lib.w4_pack_codes(FAKE, N, K, FAKE, None),
+        "w4_unpack": lambda: lib.w4_unpack(FAKE, N, K, FAKE, None),
+        "w4_gemv": lambda: lib.w4_gemv(FAKE, FAKE, FAKE, N, K, FAKE, 1, FAKE, 0, None),
+        "w4_gemv_g32": lambda: lib.w4_gemv_g32(FAKE, FAKE, FAKE, N, K, FAKE, 1, FAKE, 0, None),
+        "w4a8_gemv": lambda: lib.w4a8_gemv(FAKE, FAKE, FAKE, N, K, FAKE, FAKE, FAKE, 1, FAKE, 0,
+                                           None),
+        "w4a8_gemv_bf16": lambda: lib.w4a8_gemv_bf16(FAKE, FAKE, FAKE, N, K, FAKE, 1, FAKE, 0,
+                                                     None),
+        "q8_quantize_act": lambda: lib.q8_quantize_act(FAKE, M, K, FAKE, FAKE, FAKE, None),
+        "w4a8_mmq": lambda: lib.w4a8_mmq(FAKE, FAKE, FAKE, N, K, FAKE, FAKE, FAKE, M, FAKE, 0,
+                                         FAKE if ws else None, ws, None),
+        "w4a8_mmq_static": lambda: lib.w4a8_mmq_static(FAKE, FAKE, FAKE, N, K, FAKE, FAKE, FAKE,
+                                                       M, FAKE, 0, None),
+    }
+    for name, call in calls.items():
+        assert call() in (L.W4_ERR_CUDA, L.W4_ERR_UNSUPPORTED_DEVICE), name
