@@ -26,6 +26,8 @@ def cuda_or_skip():
 def errors(y: np.ndarray, ref: np.ndarray):
     y = np.asarray(y, np.float64)
     ref = np.asarray(ref, np.float64)
+    # equal shapes: broadcasting must never stand in for an element-wise match
+    assert y.shape == ref.shape, f"shape {y.shape} against the oracle's {ref.shape}"
     scale = np.abs(ref).max()
     max_rel = np.abs(y - ref).max() / scale if scale > 0 else np.abs(y).max()
     den = (ref ** 2).sum()
