@@ -190,8 +190,10 @@ size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K);
  *                        + m[n][g] * sum_{b in g} dx[t][b] * S[t][b] )
  * scales applied in fp32.  codes/d/m: W[N][K] planes; qa/dx/bsum: the
  * output of q8_quantize_act for x [M][K]; y: [M][N] of out_dtype.
- * M >= 1, N >= 1, K >= 256, K % 256 == 0.  `workspace` must hold
- * w4a8_mmq_workspace_size(M, N, K) bytes. */
+ * 1 <= M <= 2^24, 1 <= N <= 2^24, 256 <= K <= 131072 (512 groups),
+ * K % 256 == 0; larger sizes give W4_ERR_SHAPE.  `workspace` (16-byte
+ * aligned) must hold w4a8_mmq_workspace_size(M, N, K) bytes, else
+ * W4_ERR_WORKSPACE; it may be NULL when that size is 0. */
 int w4a8_mmq(const uint8_t *codes, const uint16_t *d_f16,
              const uint16_t *m_f16, int64_t N, int64_t K, const int8_t *qa,
              const float *dx, const int32_t *bsum, int64_t M, void *y,
