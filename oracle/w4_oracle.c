@@ -197,7 +197,11 @@ int oracle_w4_pack_grouped(const float *w, int64_t N, int64_t K, int64_t group,
                 if (wg[i] < mn) mn = wg[i];
                 if (wg[i] > mx) mx = wg[i];
             }
+#ifdef ORACLE_MUTANT_RANGE_NO_MIN
+            float range = mx;
+#else
             float range = mx - mn;
+#endif
             uint16_t d16 = float_to_f16_bits(range / 15.0f);
             uint16_t m16 = float_to_f16_bits(mn);
             float df = f16_bits_to_float(d16), mf = f16_bits_to_float(m16);
@@ -248,7 +252,11 @@ int oracle_q8_quantize(const uint16_t *x, int64_t M, int64_t K, int8_t *qa,
                 float a = fabsf(bf16_bits_to_float(xb[i]));
                 if (a > amax) amax = a;
             }
+#ifdef ORACLE_MUTANT_SCALE_128
+            float scale = amax / 128.0f;
+#else
             float scale = amax / 127.0f;
+#endif
             int32_t sum = 0;
             for (int i = 0; i < ORACLE_BLOCK; ++i) {
                 int8_t c = 0;
@@ -425,7 +433,12 @@ int oracle_mmq_rows(const uint8_t *codes, const uint16_t *d, const uint16_t *m,
 #ifdef ORACLE_MUTANT_MMQ_DROP_BLOCKSUM
                     s = 0.0;
 #endif
-                    acc += (double)dx[t * B + b] * (dd * (double)p + mm * s);
+#ifdef ORACLE_MUTANT_MMQ_NEXT_BLOCK_SCALE
+                    const int64_t bs = (bi + 1 < BPG) ? b + 1 : b;
+#else
+                    const int64_t bs = b;
+#endif
+                    acc += (double)dx[t * B + bs] * (dd * (double)p + mm * s);
                 }
             }
             y[t * W + (n - n0)] = acc;

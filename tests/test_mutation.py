@@ -4,7 +4,9 @@ Each variant is the oracle source compiled with one ``-DORACLE_MUTANT_*``
 macro (a swapped nibble order, a dropped min term, ties rounded away from
 zero, an off-by-one block sum, a shifted group index, a product that indexes
 d and m by 256-wide groups whatever the group size, a dropped block-sum term
-in the W4A8 product).  The mistake lives in the oracle on the CPU; no GPU
+in the W4A8 product, a weight scale from the maximum alone instead of the
+range, an activation scale of amax/128, and a W4A8 product that takes each
+block's scale from the next block).  The mistake lives in the oracle on the CPU; no GPU
 code is involved.  Every variant must fail at least one pin.
 """
 import pytest
@@ -20,6 +22,9 @@ MUTANTS = [
     "GROUP_INDEX",
     "GROUP_FIXED_256",
     "MMQ_DROP_BLOCKSUM",
+    "RANGE_NO_MIN",
+    "SCALE_128",
+    "MMQ_NEXT_BLOCK_SCALE",
 ]
 
 
