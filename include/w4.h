@@ -205,24 +205,29 @@ int w4a8_mmq(const uint8_t *codes, const uint16_t *d_f16,
 /* The W4A8 product of w4a8_mmq for callers that cannot allocate device memory
  * (the pages have no counterpart: this entry point exists for the library's
  * users, not for the method).  Some callers cannot call cudaMalloc or hand out
- * a workspace: code that runs while a CUDA graph is being captured, plugins
- * whose host framework owns every allocation, and deployments with a fixed
- * memory plan decided before the first request.  This entry point takes the
- * same inputs and output as w4a8_mmq but no workspace: the split-K scratch is a
- * static device array owned by the library, W4A8_MMQ_STATIC_SCRATCH_BYTES
- * (40 MiB) on every GPU that loads libw4, kept until the process exits.
+ * a workspace: plugins whose host framework owns every device allocation and
+ * gives the plugin only its inputs and outputs, and deployments whose memory
+ * plan is fixed before the first request, where an allocation in the middle
+ * of serving is not allowed.  This entry point takes the same inputs and
+ * output as w4a8_mmq but no workspace: the split-K scratch is a static device
+ * array owned by the library, W4A8_MMQ_STATIC_SCRATCH_BYTES (40 MiB) on every
+ * GPU that loads libw4, held until the process exits.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- *   - A shape whose scratch need (w4a8_mmq_workspace_size) exceeds the static
- *     size is rejected with W4_ERR_WORKSPACE before anything is enqueued (use
- *     w4a8_mmq with a caller workspace for it).
+ *   - Arguments are checked exactly as w4a8_mmq checks them, in the same
+ *     order; then a shape whose scratch need (w4a8_mmq_workspace_size)
+ *     exceeds the static size is rejected with W4_ERR_WORKSPACE before
+ *     anything is enqueued (w4a8_mmq with a caller workspace takes it).
  *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it: make
- *     that first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and caches it for the
+ *     life of the process: make that first call before any stream capture.
+ *     A device reset (cudaDeviceReset, or a reset of the primary context)
+ *     invalidates the cached address; do not call this entry point after one.
  *   - Every call on a device shares the one array and it keeps the last call's
  *     contents (the arrival counters it needs at zero are cleared on the call's
  *     stream): calls that can overlap on the GPU -- on different streams, or
  *     from several host threads -- race on it and must be serialised.
- * Arguments, layouts and results are those of w4a8_mmq. */
+ * Arguments, layouts and results are those of w4a8_mmq; for the same inputs
+ * the output is bitwise that of w4a8_mmq. */
 int w4a8_mmq_static(const uint8_t *codes, const uint16_t *d_f16,
                     const uint16_t *m_f16, int64_t N, int64_t K,
                     const int8_t *qa, const float *dx, const int32_t *bsum,

@@ -170,7 +170,11 @@ int oracle_unpack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *q) {
  *         clamp(rint((w - float(m16)) / float(d16)), 0, 15)   (ties to even)
  * so that w is approximated by float(d16)*q + float(m16), the dequantisation
  * rule w = d*q + m of the format.  Using the fp16-rounded d and m inside the
- * code computation keeps codes consistent with what is stored. */
+ * code computation keeps codes consistent with what is stored.
+ * A group minimum or maximum that equals zero is taken as +0: -0 and +0 are
+ * equal, so which of them a min/max search returns depends on where they sit
+ * in the group; storing +0 makes d and m a function of the group's values
+ * alone, independent of element order. */
 static unsigned weight_code(float w, float df, float mf) {
     if (df == 0.0f) return 0;
     float num = w - mf;
@@ -197,6 +201,10 @@ int oracle_w4_pack_grouped(const float *w, int64_t N, int64_t K, int64_t group,
                 if (wg[i] < mn) mn = wg[i];
                 if (wg[i] > mx) mx = wg[i];
             }
+#ifndef ORACLE_MUTANT_SIGNED_ZERO
+            if (mn == 0.0f) mn = 0.0f; /* -0 -> +0 */
+            if (mx == 0.0f) mx = 0.0f;
+#endif
 #ifdef ORACLE_MUTANT_RANGE_NO_MIN
             float range = mx;
 #else

@@ -136,3 +136,23 @@ def quantized_weights_direct(N: int, K: int, seed: int, group: int = GROUP):
     d = uniform_f16_bits((N, K // group), 0.001, 0.02, rng)
     m = uniform_f16_bits((N, K // group), -0.1, 0.0, rng)
     return codes, d, m
+
+def signed_zero_groups(group: int) -> np.ndarray:
+    """fp32 rows of one weight group each whose minimum or maximum is zero,
+    with -0.0 at different positions (first, middle, last, all, every other
+    slot) and ramps that end or start on -0.0: the inputs on which a min/max
+    search can return either zero."""
+    rows = []
+    z = np.zeros(group, np.float32)
+    a = z.copy(); a[0] = -0.0; rows.append(a)
+    a = z.copy(); a[group // 2] = -0.0; rows.append(a)
+    a = z.copy(); a[-1] = -0.0; rows.append(a)
+    rows.append(np.full(group, -0.0, np.float32))
+    a = z.copy(); a[1::2] = -0.0; rows.append(a)
+    a = np.linspace(0.0, 0.5, group).astype(np.float32); a[0] = -0.0; rows.append(a)
+    a = np.linspace(0.0, 0.5, group).astype(np.float32)[::-1].copy(); a[-1] = -0.0
+    rows.append(a)
+    a = np.linspace(-0.5, 0.0, group).astype(np.float32); a[-1] = -0.0; rows.append(a)
+    a = np.linspace(-0.5, 0.0, group).astype(np.float32)[::-1].copy(); a[0] = -0.0
+    rows.append(a)
+    return np.stack(rows)

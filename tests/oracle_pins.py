@@ -136,6 +136,31 @@ def pin_wpack_error_bound(o):
     assert np.all(q.reshape(N, G, GROUP).max(axis=2) == 15)
 
 
+def _check_signed_zero(o, group):
+    w = synth.signed_zero_groups(group)
+    codes, d, m = o.w4_pack(w, group=group)
+    # a zero minimum is stored as +0, whatever the position of the -0
+    mf = synth.f16_bits_to_f32(m)
+    assert np.all(m[mf == 0] == 0), m[:, 0].tolist()
+    # the same values in another order give the same d and m: flip each row
+    codes2, d2, m2 = o.w4_pack(w[:, ::-1].copy(), group=group)
+    assert np.array_equal(d, d2) and np.array_equal(m, m2)
+    # groups of zeros alone: d = +0, m = +0, codes 0
+    assert np.all(d[:5] == 0) and np.all(m[:5] == 0) and np.all(codes[:5] == 0)
+    # zero maximum with a negative minimum: d from the range, m = the minimum
+    assert synth.f16_bits_to_f32(m)[7, 0] == np.float32(-0.5)
+    assert synth.f16_bits_to_f32(d)[7, 0] == synth.f16_bits_to_f32(
+        synth.f32_to_f16_bits(np.float32(0.5) / np.float32(15.0)))
+
+
+def pin_wpack_signed_zero(o):
+    _check_signed_zero(o, GROUP)
+
+
+def pin_g32_wpack_signed_zero(o):
+    _check_signed_zero(o, 32)
+
+
 # --------------------------------------------------------------------------
 # activation quantiser
 # --------------------------------------------------------------------------

@@ -91,6 +91,16 @@ def test_pack_special_groups(torch, w4, orc):
         assert np.array_equal(g, e), name
 
 
+def test_pack_signed_zero_groups(torch, w4, orc):
+    # 32-groups whose minimum or maximum is a zero, -0 at every position
+    w = synth.signed_zero_groups(G32)
+    for ww in (w, w[:, ::-1].copy()):
+        got = _pack_gpu(torch, w4, ww)
+        want = orc.w4_pack(ww, group=G32)
+        for g, e, name in zip(got, want, ("codes", "d", "m")):
+            assert np.array_equal(g, e), name
+
+
 def test_pack_bit_exact_full_size(torch, w4, orc):
     N, K = synth.GEMV_SHAPES[2]  # 19456 x 2560
     w = synth.dense_weights(N, K, seed=synth.weight_seed(synth.CONFIG_BATCH1, 2) + 32)

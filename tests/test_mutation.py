@@ -5,8 +5,9 @@ macro (a swapped nibble order, a dropped min term, ties rounded away from
 zero, an off-by-one block sum, a shifted group index, a product that indexes
 d and m by 256-wide groups whatever the group size, a dropped block-sum term
 in the W4A8 product, a weight scale from the maximum alone instead of the
-range, an activation scale of amax/128, and a W4A8 product that takes each
-block's scale from the next block).  The mistake lives in the oracle on the CPU; no GPU
+range, an activation scale of amax/128, a W4A8 product that takes each
+block's scale from the next block, and a weight quantiser that stores a -0
+group minimum as found instead of +0).  The mistake lives in the oracle on the CPU; no GPU
 code is involved.  Every variant must fail at least one pin.
 """
 import pytest
@@ -25,6 +26,7 @@ MUTANTS = [
     "RANGE_NO_MIN",
     "SCALE_128",
     "MMQ_NEXT_BLOCK_SCALE",
+    "SIGNED_ZERO",
 ]
 
 

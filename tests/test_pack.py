@@ -53,6 +53,17 @@ def test_pack_special_groups(torch, w4, orc):
         assert np.array_equal(g, e), name
 
 
+def test_pack_signed_zero_groups(torch, w4, orc):
+    # groups whose minimum or maximum is a zero, -0 at every position: the
+    # stored d and m bits must not depend on where the -0 sits
+    w = synth.signed_zero_groups(256)
+    for ww in (w, w[:, ::-1].copy()):
+        got = _pack_gpu(torch, w4, ww)
+        want = orc.w4_pack(ww)
+        for g, e, name in zip(got, want, ("codes", "d", "m")):
+            assert np.array_equal(g, e), name
+
+
 @pytest.mark.parametrize("shape_index", range(len(synth.GEMV_SHAPES)))
 def test_pack_bit_exact_full_size(torch, w4, shape_index):
     N, K = synth.GEMV_SHAPES[shape_index]

@@ -49,6 +49,25 @@ def test_quant_special_blocks(torch, w4, orc):
     _check(torch, w4, orc, synth.f32_to_bf16_bits(x))
 
 
+def test_quant_subnormal_scales(torch, w4, orc):
+    # blocks whose dx = amax / 127 is subnormal (amax below 127 * 2^-126), so
+    # that 1 / dx overflows: amax near 1e-38, amax at the smallest normal, and
+    # blocks made only of bf16 subnormals (bf16 shares fp32's exponent range)
+    rng = np.random.default_rng(41)
+    x = np.zeros((4, 256), np.float32)
+    x[0, :32] = rng.uniform(-1e-38, 1e-38, 32)
+    x[0, 0] = 1e-38
+    x[0, 32:64] = rng.uniform(-1.0, 1.0, 32) * np.float32(2.0 ** -126)
+    x[1, :32] = np.float32(2.0 ** -126) * 127.0 * rng.uniform(-1, 1, 32)   # dx just normal
+    x[1, 32:64] = np.float32(2.0 ** -126) * 126.0 * rng.uniform(-1, 1, 32)  # dx just subnormal
+    sub = (rng.integers(1, 128, (2, 256)) * np.where(rng.random((2, 256)) < 0.5, -1, 1))
+    x[2:4] = sub.astype(np.float32) * np.float32(2.0 ** -133)             # bf16 subnormals
+    x[3, 64:96] = -0.0
+    bits = synth.f32_to_bf16_bits(x)
+    assert np.any(synth.bf16_bits_to_f32(bits[2]) != 0)
+    _check(torch, w4, orc, bits)
+
+
 @pytest.mark.parametrize("M,K", [(2048, 2560), (2048, 9728)])
 def test_quant_bit_exact_full_size(torch, w4, orc, M, K):
     _check(torch, w4, orc, synth.outlier_activations(M, K, seed=synth.act_seed(

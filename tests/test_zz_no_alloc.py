@@ -1,8 +1,10 @@
 """w4a8_mmq_static, the entry point for callers that cannot allocate device
-memory (graph-captured code, plugins whose host framework owns every
-allocation, fixed-memory deployments): it must give the same product as
-w4a8_mmq with a caller workspace, call after call, while using only the
-library's static scratch.  This file is collected last on purpose."""
+memory (plugins whose host framework owns every device allocation,
+deployments with a memory plan fixed before serving): it must give the same
+product as w4a8_mmq with a caller workspace -- bit for bit, since both run the
+same kernel with the same split count and a fixed-order split-K sum -- call
+after call, while using only the library's static scratch.  This file is
+collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -59,7 +61,11 @@ def test_static_scratch_matches_workspace_entry_point(torch, lib, orc):
                                  _ptr(S), M, _ptr(y), _lib.W4_OUT_F32, stream)
         assert rc == _lib.W4_OK, (call, _lib.status_string(rc))
         torch.cuda.synchronize()
-        parity.assert_f32_gate(y.cpu().numpy(), ref_np, f"static scratch, call {call}")
+        got = y.cpu().numpy()
+        # bitwise: a stale or mixed-up partial from the previous call's scratch
+        # contents would hide under a tolerance
+        assert np.array_equal(got.view(np.uint32), ref_np.view(np.uint32)), f"call {call}"
+        parity.assert_f32_gate(got, ref_np, f"static scratch, call {call}")
     assert lib.w4_check_device_error() == _lib.W4_OK
 
 

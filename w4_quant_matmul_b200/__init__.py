@@ -341,7 +341,10 @@ def w4a8_mmq_static(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, stream=No
     """The W4A8 product without a workspace, for callers that cannot allocate
     device memory: the split-K scratch is the library's static device array
     (shared by every call on the device; overlapping calls must be serialised).
-    Raises W4Error (W4_ERR_WORKSPACE) for shapes whose scratch need exceeds it."""
+    Raises W4Error (W4_ERR_WORKSPACE) for shapes whose scratch need exceeds it.
+    The C entry point allocates nothing; this wrapper allocates only the output
+    (through torch) when `y` is omitted, so a caller that cannot allocate
+    passes its own `y`."""
     M, K = _int8_acts(qa, dx, bsum)
     N = _weights(codes, d, m, K)
     oc = _out_code(out_dtype, y)

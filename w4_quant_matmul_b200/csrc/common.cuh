@@ -153,13 +153,22 @@ __device__ __forceinline__ bool elect_one() {
 // the reciprocal product (P. Markstein, IBM J. Res. Dev. 1990): q = q0 +
 // (x - q0 dx) rcp is within an ulp of fl(x / dx), so its rounding to an
 // integer is that of fl(x / dx) unless q lies within 2^-14 of a half-integer,
-// where the IEEE division itself decides.  Shared by the quantiser and the
-// GEMV that quantises its activations in place, so both give the same codes.
+// where the IEEE division itself decides.  A subnormal dx (block amax below
+// 127 * 2^-126) can make 1 / dx overflow to infinity, and the residual
+// x - q0 dx then falls below the normal range; every element of such a block
+// takes the IEEE division (the test is uniform across the block).  Shared by
+// the quantiser and the GEMV that quantises its activations in place, so both
+// give the same codes.
 __device__ __forceinline__ int q8_code(float x, float dx, float rcp) {
-    const float q0 = x * rcp;
-    const float q = fmaf(fmaf(-q0, dx, x), rcp, q0);
-    float qf = rintf(q);
-    if (fabsf(fabsf(q - qf) - 0.5f) < 0x1p-14f) qf = rintf(__fdiv_rn(x, dx));
+    float qf;
+    if (dx < 0x1p-126f) {
+        qf = rintf(__fdiv_rn(x, dx));
+    } else {
+        const float q0 = x * rcp;
+        const float q = fmaf(fmaf(-q0, dx, x), rcp, q0);
+        qf = rintf(q);
+        if (fabsf(fabsf(q - qf) - 0.5f) < 0x1p-14f) qf = rintf(__fdiv_rn(x, dx));
+    }
     return (int)fminf(fmaxf(qf, -127.0f), 127.0f);
 }
 

@@ -824,9 +824,15 @@ size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K) {
     return workspace_for(M, N, K, pick_splits(M, N, K, w4::sm_count()));
 }
 
-int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
-             int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
-             void* y, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Host checks shared by w4a8_mmq and w4a8_mmq_static, in one order, so that
+// both report the same status for the same bad argument.
+int validate_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
+                 int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
+                 const void* y, int out_dtype) {
     if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
     if (K / 256 > kMaxGroups || M > (1 << 24) || N > (1 << 24)) return W4_ERR_SHAPE;
     if (out_dtype != W4_OUT_BF16 && out_dtype != W4_OUT_F32) return W4_ERR_SHAPE;
@@ -834,7 +840,17 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     if (!w4::aligned16(codes) || !w4::aligned16(d_f16) || !w4::aligned16(m_f16) ||
         !w4::aligned16(qa) || !w4::aligned16(dx) || !w4::aligned16(bsum) || !w4::aligned16(y))
         return W4_ERR_ALIGN;
-    int rc = w4::check_device();
+    return w4::check_device();
+}
+
+}  // namespace
+
+extern "C" {
+
+int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
+             int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
+             void* y, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+    int rc = validate_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype);
     if (rc != W4_OK) return rc;
     int* err = w4::device_error_word();
     if (!err) return W4_ERR_CUDA;
@@ -941,8 +957,7 @@ extern "C" int w4a8_mmq_static(const uint8_t* codes, const uint16_t* d_f16,
                                const uint16_t* m_f16, int64_t N, int64_t K, const int8_t* qa,
                                const float* dx, const int32_t* bsum, int64_t M, void* y,
                                int out_dtype, void* stream) {
-    if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return W4_ERR_SHAPE;
-    int rc = w4::check_device();
+    int rc = validate_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype);
     if (rc != W4_OK) return rc;
     const size_t need = w4a8_mmq_workspace_size(M, N, K);
     if (need > (size_t)W4A8_MMQ_STATIC_SCRATCH_BYTES) return W4_ERR_WORKSPACE;

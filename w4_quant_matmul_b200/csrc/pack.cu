@@ -61,7 +61,11 @@ __global__ void __launch_bounds__(256) w4_pack_kernel(const float* __restrict__ 
             mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
         }
-        if (mn == 0.0f) mn = 0.0f;  // a zero minimum is stored as +0
+        // a zero minimum or maximum is taken as +0, so that d and m do not
+        // depend on where a -0 sits in the group (fminf/fmaxf may return
+        // either zero)
+        if (mn == 0.0f) mn = 0.0f;
+        if (mx == 0.0f) mx = 0.0f;
         const __half d16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), 15.0f));
         const __half m16 = __float2half_rn(mn);
         const float df = __half2float(d16), mf = __half2float(m16);
