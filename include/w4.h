@@ -37,6 +37,13 @@
  *     w4_check_device_error() reads (and clears) that word.
  *   - Results are bitwise deterministic run to run (fixed reduction orders, no
  *     floating-point atomics).
+ *   - The decode GEMVs (w4_gemv, w4a8_gemv, w4a8_gemv_bf16) are launched with
+ *     programmatic dependent launch and stream their weight planes without
+ *     waiting for the kernel launched immediately before them on the same
+ *     stream (their activations are read only after it has completed).  The
+ *     weight planes must therefore not be written by that immediately
+ *     preceding kernel: pack weights in an earlier launch, or put an event,
+ *     a synchronisation or any other launch in between.
  */
 #ifndef W4_H
 #define W4_H
@@ -232,6 +239,37 @@ int w4a8_mmq_static(const uint8_t *codes, const uint16_t *d_f16,
                     const uint16_t *m_f16, int64_t N, int64_t K,
                     const int8_t *qa, const float *dx, const int32_t *bsum,
                     int64_t M, void *y, int out_dtype, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Test entry points: they check the library's own machinery, not the method */
+/* ------------------------------------------------------------------------ */
+
+/* w4a8_mmq that also returns the exact integer block products it formed:
+ *   blockdots[t][n][b] = P[t][n][b] = sum_{k in block b} q[n][k] * qa[t][k]
+ * (int32 [M][N][K/32], row-major; bd_bytes >= M*N*(K/32)*4, else
+ * W4_ERR_WORKSPACE), read back from the tensor-memory accumulators of the
+ * same kernel and tiling that w4a8_mmq runs (the test instantiation of that
+ * kernel, which additionally stores every accumulator word it reads), so that
+ * the integer core can be compared with the CPU bit for bit, the practice of
+ * the GFX1100-TG150 spec ("Design": the keep-quant integer core stays
+ * bit-exact against the CPU).  y, workspace and every other argument and error
+ * are those of w4a8_mmq.  For tests: the block-product stores make it much
+ * slower than w4a8_mmq. */
+int w4a8_mmq_blockdots(const uint8_t *codes, const uint16_t *d_f16,
+                       const uint16_t *m_f16, int64_t N, int64_t K,
+                       const int8_t *qa, const float *dx, const int32_t *bsum,
+                       int64_t M, void *y, int out_dtype, int32_t *blockdots,
+                       size_t bd_bytes, void *workspace, size_t ws_bytes,
+                       void *stream);
+
+/* Runs the bounded-wait routine that every pipelined kernel of this library
+ * uses, on a wait that can never complete: one thread waits on an mbarrier
+ * phase that nothing completes, for limit_ns nanoseconds of GPU global time,
+ * then raises the device error word and returns (no trap, no fault: the
+ * context stays usable).  A following w4_check_device_error() returns
+ * W4_ERR_TIMEOUT and clears the word.  0 < limit_ns <= 100000000 (0.1 s),
+ * else W4_ERR_SHAPE.  Enqueued on `stream`. */
+int w4_test_wait_expiry(uint64_t limit_ns, void *stream);
 
 #ifdef __cplusplus
 }

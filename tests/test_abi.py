@@ -119,6 +119,13 @@ def test_pack_and_quantizer_validation(lib):
     assert lib.q8_quantize_act(FAKE, 0, 64, FAKE, FAKE, FAKE, None) == L.W4_OK
 
 
+def test_wait_expiry_validation(lib):
+    # limits outside (0, 0.1 s] are refused before any device work
+    from w4_quant_matmul_b200 import _lib as L
+    assert lib.w4_test_wait_expiry(0, None) == L.W4_ERR_SHAPE
+    assert lib.w4_test_wait_expiry(100_000_001, None) == L.W4_ERR_SHAPE
+
+
 def test_mmq_validation(lib):
     from w4_quant_matmul_b200 import _lib as L
     f = lib.w4a8_mmq

@@ -18,8 +18,10 @@ KNOWN_SPILLS = {
     "w4_gemv_rows_kernel<4, 2, 4, 0, 3>": 12,
     # the same for group-32 weights
     "w4_gemv_rows_kernel<4, 2, 4, 0, 0>": 4,
-    # the W4A8 prefill kernel (one kernel, warp-specialised with setmaxnreg)
-    "w4a8_mmq_kernel(": 16,
+    # the W4A8 prefill kernel (warp-specialised with setmaxnreg) and its test
+    # instantiation that also stores the block products
+    "w4a8_mmq_kernel<false>(": 16,
+    "w4a8_mmq_kernel<true>(": 12,
 }
 
 
@@ -76,3 +78,18 @@ def test_parser_sees_a_spill():
             "ptxas info    : Function properties for _Z3foov\n"
             "    8 bytes stack frame, 4 bytes spill stores, 4 bytes spill loads\n")
     assert _spills(text) == {"_Z3foov": 4}
+
+
+def test_build_flags_keep_denormals_and_ieee_division():
+    # The W4A8 product's epilogue reads exact integer products as fp32
+    # denormals (V * 2^-149) and multiplies them at full rate; flushing
+    # denormals to zero would silently zero every product.  The quantisers
+    # rely on IEEE division and rounding.  So no fast-math-style flag may
+    # reach nvcc.
+    from w4_quant_matmul_b200 import build
+    flags = " ".join(build.NVCC_FLAGS)
+    for bad in ("--use_fast_math", "-use_fast_math", "-ftz=true", "--ftz=true",
+                "-prec-div=false", "--prec-div=false", "-prec-sqrt=false",
+                ):
+        assert bad not in flags, bad
+

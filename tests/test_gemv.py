@@ -92,12 +92,16 @@ def test_activation_outliers_and_dynamic_range(torch, w4, orc):
 
 
 @pytest.mark.parametrize("shape_index", range(len(synth.GEMV_SHAPES)))
-def test_full_size_sampled_rows(torch, w4, orc, shape_index):
+def test_full_size(torch, w4, orc, shape_index):
     N, K = synth.GEMV_SHAPES[shape_index]
     _, codes, d, m = parity.packed_dense_weights(N, K, synth.weight_seed(synth.CONFIG_BATCH1,
                                                                          shape_index))
-    rows = parity.sample_rows(N)
+    # every row at M = 1 on all five shapes and at M = 8 on the four layer
+    # shapes (every row block of the launch the benchmark times); a seeded
+    # sample of rows (both ends + 256 interior) otherwise
+    sampled = parity.sample_rows(N)
     for M in (1, 2, 4, 8):
+        rows = None if (M == 1 or (M == 8 and shape_index < 4)) else sampled
         cfg = synth.CONFIG_BATCH1 if M == 1 else synth.CONFIG_SMALL_BATCH
         x = synth.activations(M, K, synth.act_seed(cfg, shape_index))
         _both(torch, w4, orc, codes, d, m, x, rows=rows, what=f"{N}x{K} M{M}")

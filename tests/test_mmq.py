@@ -159,3 +159,51 @@ def test_pipeline_with_gpu_quantiser(torch, w4, orc):
     torch.cuda.synchronize()
     ref = orc.mmq(codes, d, m, *orc.q8_quantize(x))
     parity.assert_f32_gate(y.cpu().numpy(), ref, "gpu quantiser -> mmq")
+
+
+@pytest.mark.parametrize("M,N,K", [(130, 200, 768), (257, 129, 512), (64, 384, 4096),
+                                   (300, 260, 2560), (256, 384, 9728)])
+def test_integer_block_products_bit_exact(torch, w4, orc, M, N, K):
+    # The exact int32 block products P[t][n][b], read back from the tensor
+    # memory of the same kernel (its test instantiation), equal the oracle's
+    # int64 products element for element: ragged M and N, several groups, and
+    # (K = 9728 at M = 256) the split-K path.  The y of the same call meets the
+    # float gate.
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=7 * M + N + K)
+    qa, dx, S = orc.q8_quantize(synth.outlier_activations(M, K, seed=M + 3 * N + K))
+    dev = (torch.from_numpy(codes).cuda(), _dev_u16(torch, d, torch.float16),
+           _dev_u16(torch, m, torch.float16), torch.from_numpy(qa).cuda(),
+           torch.from_numpy(dx).cuda(), torch.from_numpy(S).cuda())
+    y, P = w4.w4a8_mmq_blockdots(*dev, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    want = orc.mmq_blockdots(codes, qa)
+    got = P.cpu().numpy().astype(np.int64)
+    bad = int((got != want).sum())
+    assert bad == 0, f"{bad} of {want.size} block products differ"
+    parity.assert_f32_gate(y.cpu().numpy(), orc.mmq(codes, d, m, qa, dx, S), f"M{M} N{N} K{K}")
+    # the product entry point gives the same y bit for bit
+    y2 = w4.w4a8_mmq(*dev, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+
+
+def test_integer_block_products_extreme(torch, w4, orc):
+    # every block at the ends of the integer range, +-32*15*127
+    M, N, K = 128, 128, 512
+    codes = np.full((N, K // 2), 0xFF, np.uint8)
+    d = synth.f32_to_f16_bits(np.full((N, K // 256), 0.01, np.float32))
+    m = synth.f32_to_f16_bits(np.full((N, K // 256), -0.05, np.float32))
+    qa = np.full((M, K), 127, np.int8)
+    qa[64:96] = -127
+    qa[96:, ::2] = -127
+    dx = np.full((M, K // 32), 0.01, np.float32)
+    S = qa.astype(np.int32).reshape(M, K // 32, 32).sum(axis=2).astype(np.int32)
+    dev = (torch.from_numpy(codes).cuda(), _dev_u16(torch, d, torch.float16),
+           _dev_u16(torch, m, torch.float16), torch.from_numpy(qa).cuda(),
+           torch.from_numpy(dx).cuda(), torch.from_numpy(S).cuda())
+    _, P = w4.w4a8_mmq_blockdots(*dev, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    want = orc.mmq_blockdots(codes, qa)
+    assert want.max() == 60960 and want.min() == -60960
+    assert np.array_equal(P.cpu().numpy().astype(np.int64), want)
+

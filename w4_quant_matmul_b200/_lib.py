@@ -45,6 +45,9 @@ SIGNATURES = {
     "w4a8_mmq": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P, ctypes.c_size_t, _P],
                  _INT),
     "w4a8_mmq_static": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P], _INT),
+    "w4_test_wait_expiry": ([ctypes.c_uint64, _P], _INT),
+    "w4a8_mmq_blockdots": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P,
+                            ctypes.c_size_t, _P, ctypes.c_size_t, _P], _INT),
 }
 
 W4A8_MMQ_STATIC_SCRATCH_BYTES = 40 * 1024 * 1024

@@ -23,6 +23,10 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libw4.so")
 SOURCES = ["abi.cu", "pack.cu", "quant.cu", "gemv.cu", "mmq.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# No --use_fast_math / -ftz=true / -prec-div=false: the W4A8 product's epilogue
+# multiplies exact integer products held as fp32 denormals, which a
+# flush-to-zero build would zero, and the quantisers depend on IEEE division
+# and rounding (tests/test_build_audit.py checks these flags).
 NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
                      "-Xptxas", "-v", "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
 

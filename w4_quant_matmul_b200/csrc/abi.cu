@@ -8,6 +8,8 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
+// Longest wait w4_test_wait_expiry accepts (0.1 s).
+constexpr uint64_t kMaxTestWaitNs = 100000000ull;
 
 // One error word per device; kernels raise W4_ERR_TIMEOUT here when a bounded
 // wait runs out.
@@ -25,6 +27,20 @@ int current_device(int* dev) {
     if (e != cudaSuccess) return w4::cuda_fail(e);
     if (*dev < 0 || *dev >= kMaxDevices) return W4_ERR_UNSUPPORTED_DEVICE;
     return W4_OK;
+}
+
+// Test of the bounded-wait path: one thread waits on an mbarrier whose phase
+// nothing completes, with the caller's limit, through the same wait routine
+// every pipelined kernel uses.  When the limit runs out the routine raises the
+// device error word and the kernel returns normally.
+__global__ void wait_expiry_kernel(unsigned long long limit_ns, int* err) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    w4::mbar_init(&bar, 1);
+    abort_flag = 0;
+    w4::fence_mbar_init();
+    // phase 0 of `bar` needs one arrival that never comes
+    (void)w4::mbar_wait_for(&bar, 0u, &abort_flag, err, limit_ns);
 }
 
 }  // namespace
@@ -116,6 +132,16 @@ int w4_check_device_error(void) {
         return v;
     }
     return W4_OK;
+}
+
+int w4_test_wait_expiry(uint64_t limit_ns, void* stream) {
+    if (limit_ns == 0 || limit_ns > kMaxTestWaitNs) return W4_ERR_SHAPE;
+    int rc = w4::check_device();
+    if (rc != W4_OK) return rc;
+    int* err = w4::device_error_word();
+    if (!err) return W4_ERR_CUDA;
+    wait_expiry_kernel<<<1, 1, 0, (cudaStream_t)stream>>>((unsigned long long)limit_ns, err);
+    return w4::launch_status();
 }
 
 }  // extern "C"

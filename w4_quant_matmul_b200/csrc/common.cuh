@@ -74,8 +74,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // cut short) is raised by another thread, or after
 // kWaitLimitNs, in which case it raises the flag and the device error word.
 // Returns false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag, int* err_word) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int* err_word,
+                                              unsigned long long limit_ns) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
@@ -83,13 +84,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
         if (mbar_try_wait(a, parity)) return true;
         if ((i & 31u) == 0) {
             if (abort_flag && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 if (abort_flag) *abort_flag = 1;
                 if (err_word) atomicExch(err_word, (int)W4_ERR_TIMEOUT);
                 return false;
             }
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag, int* err_word) {
+    return mbar_wait_for(bar, parity, abort_flag, err_word, kWaitLimitNs);
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {

@@ -40,15 +40,17 @@
 //    4-stage shared-memory ring completed on mbarriers, so the whole range is
 //    in flight without registers; 16 consumer half-warps run the same inner
 //    loop, one row each, from shared memory.
-//  * Programmatic dependent launch (ring kernel).  Before griddepcontrol.wait
-//    a CTA only asks L2 to prefetch its first weights (bulk L2 prefetch; L2 is
-//    the point of coherence, so a prefetch can never observe stale data even
-//    if the preceding kernel writes the weights).  In a chain of launches the
-//    first HBM round trip of this GEMV overlaps the tail of the previous
-//    kernel; every load that feeds arithmetic happens after the wait.  The
-//    row kernel is launched in plain stream order (its dependency wait is
-//    then a no-op): measured in a five-GEMV decode step, its CTAs launched
-//    early behind a ring kernel cost more than the overlap gained.
+//  * Programmatic dependent launch (ring kernel).  The producer lane reads
+//    only the weight planes and never waits for the preceding kernel, so in a
+//    chain of launches this GEMV's ring fills while the previous kernel is
+//    still running; the consumers wait (griddepcontrol.wait) before they read
+//    the activations.  The weight planes must therefore not be written by the
+//    kernel launched immediately before on the same stream.  At M = 1 the ring
+//    kernel runs one CTA per SM in at most half of the SM's shared memory, so
+//    that the next kernel's CTAs fit beside it.  The row kernel is launched in
+//    plain stream order (its dependency wait is then a no-op): measured in a
+//    five-GEMV decode step, its CTAs launched early behind a ring kernel cost
+//    more than the overlap gained.
 //  * Activation forms.  The same kernels also take the activations as int8
 //    blocks of 32 (qa, dx, S from q8_quantize_act: the 32-code chunk is one
 //    block, two dp4a per code word give its exact dot product P, then
@@ -580,7 +582,7 @@ constexpr int kRingThreads = 32 * (kRingWarps + 1);     // + the producer warp
 constexpr int kRowsPerStage = 2 * kRingWarps;           // 16
 constexpr int kChunkBytes = 1280;                       // K-chunk of a row per stage
 constexpr int kStageBytes = kRowsPerStage * kChunkBytes;  // 20 KB
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 5;
 constexpr int kSmemPerSm = 227 * 1024;                  // usable per CTA on sm_100
 constexpr size_t kRingMaxCodeBytes = (size_t)16 << 20;  // streams below this use the ring
 
@@ -644,14 +646,11 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
 
     if (warp == kRingWarps) {
         // ---------------- producer: one lane streams the code ring ----------------
+        // The producer reads only the weight planes, which do not depend on
+        // the preceding kernel in the stream (the caller's contract), so it
+        // never waits for that kernel: under programmatic dependent launch the
+        // ring fills while the preceding kernel is still running.
         if (w4::elect_one()) {
-            // before the dependency wait only L2 prefetches (L2 is the point of
-            // coherence: a prefetch cannot hand stale weights to a later load)
-            const int first = min(kRowsPerStage, r1 - r0);
-            const uint32_t b0 = (uint32_t)min(kChunkBytes, row_bytes);
-            for (int r = 0; r < first; ++r)
-                l2_prefetch(codes + (size_t)(r0 + r) * row_bytes, b0);
-            pdl_wait();
             int it = 0;
             for (; it < nstage; ++it) {
                 const int s = it % stages;
@@ -837,7 +836,21 @@ struct Plan {
 
 Plan plan_for(int M, int C) {
     Plan p{0, 0, 0};
-    for (int st = kMaxStages; st >= 2; --st) {
+    if (M == 1) {
+        // one CTA per SM, at most half of the SM's shared memory, so that the
+        // next kernel's CTAs (launched early by programmatic dependent launch)
+        // fit beside this one's and fill their rings while it finishes
+        for (int st = kMaxStages; st >= 2; --st) {
+            const size_t need = layout(M, C, st).total;
+            if (need + 1024 <= (size_t)114 * 1024) {
+                p.stages = st;
+                p.smem = need;
+                p.per_sm = 1;
+                return p;
+            }
+        }
+    }
+    for (int st = 4; st >= 2; --st) {
         const size_t need = layout(M, C, st).total;
         if (need <= (size_t)kSmemPerSm) {
             p.stages = st;

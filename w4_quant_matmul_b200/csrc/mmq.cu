@@ -16,28 +16,31 @@
 //   warp 0      TMA producer: the qa tile (128 x 128 B, 128B-swizzled) and the
 //               packed code tile (128 rows x 64 B) into a 4-stage ring, and,
 //               ahead of each 256-group, that group's dx and S for the tile's
-//               128 tokens (8 x 128 boxes of fp32 / int32) into a 2-slot ring.
+//               128 tokens (8 x 128 boxes of fp32 / int32) into a 4-slot ring.
 //   warp 1      allocates 512 TMEM columns = four 128-column block buffers;
 //               one lane issues, per 32-block, a tcgen05.mma.kind::i8 (M=128,
 //               N=128, K=32; A = qa as s8, B = the codes as u8) into the
-//               buffer of the block's position in the stage, and one
+//               buffer of the block's position in the stage, as soon as the
+//               epilogue has read that buffer's previous block, and one
 //               tcgen05.commit per buffer pair.
 //   warps 2-3   unpack each code tile, nibble -> byte, into the 128B-swizzled
 //               K-major layout the MMA's shared-memory descriptor expects
-//               (tcgen05 has no 4-bit integer kind).
+//               (tcgen05 has no 4-bit integer kind), and at each group's first
+//               stage write the tile's d and m (fp32) into a 4-slot ring.
 //   warps 4-11  epilogue: each thread owns one token row (its TMEM lane) and 64
-//               weight rows; per buffer pair it waits once, reads both blocks'
-//               words and releases the pair; the thread that sees a stage's
-//               last pair also frees that stage's shared-memory operands.  d
-//               and m move per group through a 2-slot shared ring: each of the
-//               256 epilogue threads loads one of the tile's next-group values
-//               a group ahead and writes it at the group's end.  Shared memory
-//               (~190 KB) does not depend on K.
+//               weight rows.  It reads each block's words in two 32-column
+//               halves, releases every buffer as soon as its words are in
+//               registers, and frees a stage's shared-memory operands once the
+//               stage's last commit has landed.  Shared memory (~205 KB) does
+//               not depend on K.
 //
-// On B200 the tensor pipe runs MMAs and commits one after another, and a
-// commit costs about as much as 1.5 of these MMAs (measured), so commits are
-// per pair of blocks rather than per block, and the shared-memory stage is
-// released by the epilogue, not by a further commit.
+// Measured on B200 (single-SM microbenchmarks): a 128x128x32 kind::i8 MMA
+// occupies the tensor pipe 65 cycles (8000 MAC/clk, the full int8 rate), a
+// commit adds ~100 cycles when it follows short MMAs, and TMEM -> registers
+// moves ~390 B/clk/SM while the words are consumed by FMAs.  The epilogue
+// (one FMA and 4 TMEM bytes per 32 multiply-adds) therefore bounds the kernel,
+// not the tensor pipe: commits are per pair of blocks and everything else is
+// arranged so that the epilogue warps never wait.
 //
 // Epilogue arithmetic.  Converting 16384 int32 products per block to float at
 // the quarter-rate conversion throughput would cost four times the MMA, so
@@ -51,17 +54,21 @@
 // summation turns the per-block scaling into one full-rate FMA per element
 // per block with per-(token, block) coefficients:
 //   sum_b dx_b P_b = sum_{r<4} [ (dx_r - dx_{r+4}) V_r + dx_{r+4} V_{r+4} ]
-//                    - 2^17 sum_{r<4} dx_r,
-// the coefficients scaled by a power of two 2^e per (token, group) so that
-// the products stay normal.  At the group end one FMA recovers
-// acc * 2^(149-e) - 2^17 sum_{r<4} dx_r, and y += d * that + m * sum_b dx_b S_b.
-// The exact integer block sums never leave TMEM as anything but exact values;
-// the fp32 work is the coefficient differences and the accumulation.
-// Requires |dx| < 2^100 (activations far beyond any fp16/bf16 model range
-// would overflow the scaled products).
+//                    - 2^17 sum_{r<4} dx_r.
+// The coefficients carry a factor 2^e, one e per token for the whole unit,
+// chosen from the token's largest block scale so that the products stay
+// normal (dx_max 2^e in [2^40, 2^41)); a later group whose scales are 2^24
+// times larger lowers e and rescales the partial output.  The bias term
+// -2^17 sum dx_r enters as the addend of the group's first FMA, and the
+// output row is kept in units of 2^(e-149), so the group end costs two FMAs
+// per element, ys += d * acc + m * (sum_b dx_b S_b), and the unit end one
+// multiply by 2^(149-e).  The exact integer block sums never leave TMEM as
+// anything but exact values; the fp32 work is the coefficient differences and
+// the accumulation.  Requires |dx| < 2^100 (activations far beyond any
+// fp16/bf16 model range would overflow the scaled products).
 //
-// Registers are rebalanced with setmaxnreg: 48 per thread for warps 0-3, 224
-// for the epilogue (128*48 + 256*224 <= 384*168, the launch allotment).
+// Registers are rebalanced with setmaxnreg: 56 per thread for warps 0-3, 224
+// for the epilogue (128*56 + 256*224 = 384*168, the launch allotment).
 // K slices (split-K) write fp32 partial tiles to the caller's workspace; the
 // CTA that finishes a tile last sums the partials in slice order (bitwise
 // deterministic) and stores y.
@@ -85,8 +92,8 @@ constexpr int KB = 32;         // activation block = MMA K for kind::i8
 constexpr int STAGES = 4;
 constexpr int NTB = 4;         // TMEM block buffers (BN columns each)
 constexpr int NPAIR = NTB / 2; // buffer pairs: the unit of MMA -> epilogue hand-off
+constexpr int kRing = 4;       // slots of the per-group dx/S and d/m rings
 constexpr int BIAS_BYTES = 128 * KB;  // one constant operand tile of the bias MMA
-constexpr int kBiasLog2 = 17;         // accumulator bias 2^17 (see the header)
 constexpr int kThreads = 384;              // 4 producer-side warps + 8 epilogue warps
 constexpr int kEpiWarps = 8;
 constexpr int kEpiCols = BN / (kEpiWarps / 4); // 64 weight rows per epilogue thread
@@ -103,16 +110,18 @@ struct Smem {
     static constexpr int b = a + STAGES * A_BYTES;
     static constexpr int bp = b + STAGES * B_BYTES;
     static constexpr int bias = bp + STAGES * BP_BYTES;  // bias MMA operands (A, B)
-    static constexpr int bars = bias + 2 * BIAS_BYTES;   // uint64 barriers
-    static constexpr int nbars = 3 * STAGES + 2 * NPAIR + 1 + 4 + 4;
-    static constexpr int misc = bars + nbars * 8;        // tmem base, abort flag
-    static constexpr int dm = (misc + 16 + 15) & ~15;    // fp32 [2 slots][d, m][BN]
-    // ring of per-group activation scales and block sums (two slots of
-    // dx fp32 [128 tokens][8] + S int32 [128][8]), after d and m
+    // ring of per-group activation scales and block sums: per slot dx fp32
+    // [128 tokens][8] then S int32 [128][8]
     static constexpr int kScSlotBytes = 2 * BM * 8 * 4;
-    static constexpr int sc = (dm + 2 * 2 * BN * 4 + 127) & ~127;
-    static constexpr size_t total = (size_t)sc + 2 * kScSlotBytes + 1024;
+    static constexpr int sc = bias + 2 * BIAS_BYTES;
+    static constexpr int dm = sc + kRing * kScSlotBytes;  // fp32 [kRing][d, m][BN]
+    static constexpr int bars = dm + kRing * 2 * BN * 4;  // uint64 barriers
+    static constexpr int nbars = 3 * STAGES + NPAIR + NTB + 1 + 4 * kRing;
+    static constexpr int misc = bars + nbars * 8;         // tmem base, abort flag, last flag
+    static constexpr size_t total = (size_t)misc + 16 + 1024;
 };
+
+static_assert(Smem::sc % 128 == 0 && Smem::dm % 16 == 0, "ring slots must be aligned");
 
 struct Params {
     const __half* d;
@@ -128,6 +137,7 @@ struct Params {
     int units;             // tiles * splits work units (CTAs loop over them)
     int* counters;         // [tiles] arrival counters (split > 1), zeroed before launch
     float* partials;       // [tiles][splits][BM][BN] fp32 partial tiles
+    int32_t* dump;         // test instantiation only: [M][N][K/32] words read back
 };
 
 
@@ -188,14 +198,33 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_wait_ld() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 // ---------------------------------------------------------------------------
 // kernel
 // ---------------------------------------------------------------------------
 
+// Wait for tcgen05.ld results: the registers are named as operands, so that
+// the compiler cannot move their uses above the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+          "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+          "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+          "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+          "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+          "+r"(r[31])
+        :
+        : "memory");
+}
+
+__device__ __forceinline__ float pow2f(int e) {  // 2^e for -126 <= e <= 127
+    return __uint_as_float((uint32_t)(e + 127) << 23);
+}
+
+// kDump (the test instantiation behind w4a8_mmq_blockdots) also stores every
+// word read from TMEM, minus the 2^17 bias, to p.dump.
+template <bool kDump>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a8_mmq_kernel(const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_b,
@@ -208,54 +237,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* sa = smem + Smem::a;
     uint8_t* sb = smem + Smem::b;
     uint8_t* sbp = smem + Smem::bp;
+    uint8_t* sc = smem + Smem::sc;
+    float* dm_s = reinterpret_cast<float*>(smem + Smem::dm);  // [kRing][d, m][BN]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Smem::bars);
-    uint64_t* full = bars;                   // TMA landed (A + packed B)
-    uint64_t* unpacked = bars + STAGES;      // B unpacked into the MMA layout
-    uint64_t* empty = bars + 2 * STAGES;     // MMAs of the stage done (seen by the epilogue)
-    uint64_t* tfull = bars + 3 * STAGES;     // TMEM buffer pair written
-    uint64_t* tempty = tfull + NPAIR;        // TMEM buffer pair read out
-    uint64_t* drain = tempty + NPAIR;        // final MMA completion
-    uint64_t* scfull = drain + 1;            // a group's dx/S landed in its slot
-    uint64_t* scempty = scfull + 2;          // the epilogue has read the slot
-    uint64_t* dmfull = scempty + 2;          // a group's d, m written to their slot
-    uint64_t* dmfree = dmfull + 2;           // every epilogue warp has read the slot
+    uint64_t* full = bars;                   // TMA landed (A + packed B)       [STAGES]
+    uint64_t* unpacked = full + STAGES;      // B unpacked into the MMA layout  [STAGES]
+    uint64_t* sfree = unpacked + STAGES;     // the stage's MMAs are complete   [STAGES]
+    uint64_t* tfull = sfree + STAGES;        // TMEM buffer pair written        [NPAIR]
+    uint64_t* tempty = tfull + NPAIR;        // TMEM buffer read out            [NTB]
+    uint64_t* drain = tempty + NTB;          // final MMA completion
+    uint64_t* scfull = drain + 1;            // a group's dx/S landed           [kRing]
+    uint64_t* scempty = scfull + kRing;      // the epilogue has read the slot  [kRing]
+    uint64_t* dmfull = scempty + kRing;      // a group's d, m written          [kRing]
+    uint64_t* dmfree = dmfull + kRing;       // every epilogue warp has read it [kRing]
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Smem::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
     volatile int* last_flag = abort_flag + 1;
-    float* dm_s = reinterpret_cast<float*>(smem + Smem::dm);  // [2][2][BN]
     const int G = p.K / 256;
-    uint8_t* sc = smem + Smem::sc;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int ngroups = G;
 
-    // Work unit u -> (tile_m, tile_n, K slice).  Units handed to consecutive
-    // CTAs share tile_m, i.e. the same activation rows.
+    // Work unit u -> (tile_m, tile_n, K slice [gb, ge) in groups).  Units handed
+    // to consecutive CTAs share tile_m, i.e. the same activation rows.
     auto unit_of = [&](int u, int& tm, int& tn, int& gb, int& ge) {
         const int split = u % p.splits;
         const int tile = u / p.splits;
         tn = tile % p.tiles_n;
         tm = tile / p.tiles_n;
-        gb = (int)(((long long)ngroups * split) / p.splits);
-        ge = (int)(((long long)ngroups * (split + 1)) / p.splits);
+        gb = (int)(((long long)G * split) / p.splits);
+        ge = (int)(((long long)G * (split + 1)) / p.splits);
     };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             w4::mbar_init(&full[i], 1);
             w4::mbar_init(&unpacked[i], 2);
-            w4::mbar_init(&empty[i], 1);
+            w4::mbar_init(&sfree[i], 1);
         }
-        for (int i = 0; i < NPAIR; ++i) {
-            w4::mbar_init(&tfull[i], 1);
-            w4::mbar_init(&tempty[i], kEpiWarps);
-        }
+        for (int i = 0; i < NPAIR; ++i) w4::mbar_init(&tfull[i], 1);
+        for (int i = 0; i < NTB; ++i) w4::mbar_init(&tempty[i], kEpiWarps);
         w4::mbar_init(drain, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kRing; ++i) {
             w4::mbar_init(&scfull[i], 1);
             w4::mbar_init(&scempty[i], kEpiWarps);
-            w4::mbar_init(&dmfull[i], kEpiWarps);
+            w4::mbar_init(&dmfull[i], 2);
             w4::mbar_init(&dmfree[i], kEpiWarps);
         }
         *abort_flag = 0;
@@ -265,8 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every accumulator starts at 32 * 64 * 64 = 2^17
     {
         uint32_t* ba = reinterpret_cast<uint32_t*>(smem + Smem::bias);
-        for (int i = threadIdx.x; i < 2 * BIAS_BYTES / 4; i += kThreads)
-            ba[i] = 0x40404040u;
+        for (int i = threadIdx.x; i < 2 * BIAS_BYTES / 4; i += kThreads) ba[i] = 0x40404040u;
         w4::fence_proxy_async_smem();
     }
     if (warp == 1) {
@@ -282,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 48;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
         if (warp == 0) {
             // ---------------- TMA producer ----------------
             if (w4::elect_one()) {
@@ -290,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 w4::prefetch_tmap(&tm_b);
                 w4::prefetch_tmap(&tm_dx);
                 w4::prefetch_tmap(&tm_s);
-                int it = 0;  // global stage counter
+                int it = 0;  // stages issued
                 int gi = 0;  // groups whose scales were issued
                 bool ok = true;
                 for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
@@ -298,10 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     unit_of(u, tmi, tni, gb, ge);
                     for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
                         if ((kg & 1) == 0) {
-                            // the group's dx and S for the tile's 128 tokens, ahead of
-                            // its first stage (rows past M are zero-filled)
-                            const int slot = gi & 1;
-                            if (!w4::mbar_wait(&scempty[slot], ((uint32_t)(gi >> 1) & 1u) ^ 1u,
+                            // the group's dx and S for the tile's 128 tokens (rows
+                            // past M are zero-filled), into slot gi % kRing
+                            const int slot = gi % kRing;
+                            if (!w4::mbar_wait(&scempty[slot], ((uint32_t)(gi / kRing) & 1u) ^ 1u,
                                                abort_flag, p.err)) {
                                 ok = false;
                                 break;
@@ -315,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         const int s = it % STAGES;
                         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                        if (!w4::mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.err)) {
+                        if (!w4::mbar_wait(&sfree[s], ph ^ 1u, abort_flag, p.err)) {
                             ok = false;
                             break;
                         }
@@ -328,8 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // drain: every issued load must land before the CTA exits
                 for (int k = it - STAGES < 0 ? 0 : it - STAGES; k < it; ++k)
                     w4::mbar_wait(&full[k % STAGES], (uint32_t)(k / STAGES) & 1u, nullptr, p.err);
-                for (int k = gi - 2 < 0 ? 0 : gi - 2; k < gi; ++k)
-                    w4::mbar_wait(&scfull[k & 1], (uint32_t)(k >> 1) & 1u, nullptr, p.err);
+                for (int k = gi - kRing < 0 ? 0 : gi - kRing; k < gi; ++k)
+                    w4::mbar_wait(&scfull[k % kRing], (uint32_t)(k / kRing) & 1u, nullptr, p.err);
             }
         } else if (warp == 1) {
             // ---------------- MMA issuer ----------------
@@ -365,23 +390,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // seeded with the bias before its block; second half: the
                         // block accumulates onto the first half's block in that buffer.
                         const bool seed = (kg & 1) == 0;
-                        for (int j = 0; j < NPAIR && ok; ++j) {
-                            // wait until the epilogue has read this pair's previous
-                            // blocks (first use: free)
-                            if (!w4::mbar_wait(&tempty[j], ((uint32_t)it & 1u) ^ 1u, abort_flag,
-                                               p.err)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
+#pragma unroll
+                        for (int j = 0; j < NPAIR; ++j) {
 #pragma unroll
                             for (int qq = 0; qq < 2; ++qq) {
                                 const int q = 2 * j + qq;  // block in the stage = buffer
+                                // the epilogue has read this buffer's previous block
+                                if (!w4::mbar_wait(&tempty[q], ((uint32_t)it & 1u) ^ 1u,
+                                                   abort_flag, p.err)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after();
                                 const uint32_t dt = tmem_base + (uint32_t)(q * BN);
                                 if (seed) mma_i8(dt, bias_a, bias_b, idesc_bias, 0u);  // D = 2^17
                                 mma_i8(dt, smem_desc_sw128(a_addr + q * KB),
                                        smem_desc_sw128(b_addr + q * KB), idesc, 1u);  // D += P
                             }
+                            if (!ok) break;
                             mma_commit(&tfull[j]);
                         }
                     }
@@ -391,8 +417,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         } else {
             // ---------------- unpackers (warps 2, 3) ----------------
+            // Per stage: the packed code tile, nibble -> byte, into the 128B-
+            // swizzled K-major layout of the MMA's B operand.  Per group: the
+            // tile's d and m (fp16 -> fp32) into slot g % kRing of the d/m ring.
             const int ut = threadIdx.x - 64;  // 0..63
             int it = 0;
+            int gq = 0;  // groups whose d, m were written
             bool ok = true;
             for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                 int tmi, tni, gb, ge;
@@ -400,6 +430,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    const bool group_start = (kg & 1) == 0;
+                    float dmv[4];
+                    if (group_start) {
+                        // issue the group's d, m loads before the unpack: thread ut
+                        // owns entries ut + 64 i of [d, m][BN]
+                        const int g = kg >> 1;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int v = ut + 64 * i;
+                            const int n = tni * BN + (v & (BN - 1));
+                            const __half* src = (v >> 7) ? p.m : p.d;
+                            dmv[i] = n < p.N ? __half2float(src[(size_t)n * G + g]) : 0.0f;
+                        }
+                    }
                     if (!w4::mbar_wait(&full[s], ph, abort_flag, p.err)) {
                         ok = false;
                         break;
@@ -424,13 +468,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     w4::fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) w4::mbar_arrive(&unpacked[s]);
+                    if (group_start) {
+                        const int slot = gq % kRing;
+                        // the slot's previous group (gq - kRing) has been read
+                        if (!w4::mbar_wait(&dmfree[slot], ((uint32_t)(gq / kRing) & 1u) ^ 1u,
+                                           abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        float* d_dst = dm_s + slot * 2 * BN;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) d_dst[ut + 64 * i] = dmv[i];
+                        __syncwarp();
+                        if (lane == 0) w4::mbar_arrive(&dmfull[slot]);
+                        ++gq;
+                    }
                 }
             }
         }
     } else {
         // ---------------- epilogue (warps 4..11) ----------------
         asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
-        const int et = threadIdx.x - 128;           // 0..255
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
         const int cs = (warp - 4) >> 2;             // column slice: kEpiCols weight rows
         const int row = quarter * 32 + lane;        // token row within the tile
@@ -440,22 +498,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         int gi = 0;  // groups started (the slot sequence of both per-group rings)
         bool ok = true;
-        // d and m travel per group through a two-slot ring: thread et owns one
-        // value (d if et < 128, else m) of weight row (et & 127) of the tile; it
-        // loads the next group's value at a group's start and writes it to the
-        // other slot at the group's end.
-        auto dm_value = [&](int n0v, int gv) -> float {
-            const int n = n0v + (et & (BN - 1));
-            const __half* src = (et >> 7) ? p.m : p.d;
-            return n < p.N ? __half2float(src[(size_t)n * G + gv]) : 0.0f;
-        };
-        if (blockIdx.x < p.units) {
-            int tmi0, tni0, gb0, ge0;
-            unit_of(blockIdx.x, tmi0, tni0, gb0, ge0);
-            dm_s[et] = dm_value(tni0 * BN, gb0);  // slot 0 ([d, m][BN]): first group
-            __syncwarp();
-            if (lane == 0) w4::mbar_arrive(&dmfull[0]);
-        }
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             int tmi, tni, g_begin, g_end;
             unit_of(u, tmi, tni, g_begin, g_end);
@@ -463,173 +505,160 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int t = tmi * BM + row;
             const bool t_live = t < p.M;
 
-            float acc[kEpiCols], yv[kEpiCols];
+            // ys: the output row slice in units of 2^(e - 149), e per token, set
+            // from the token's activation scales (see the file header)
+            float acc[kEpiCols], ys[kEpiCols];
 #pragma unroll
-            for (int c = 0; c < kEpiCols; ++c) {
-                acc[c] = 0.0f;
-                yv[c] = 0.0f;
-            }
-            float kpow = 0.0f, neg_bias = 0.0f, tmin = 0.0f;
-            float cf[8];  // per-block coefficients of the current group, times 2^e
+            for (int c = 0; c < kEpiCols; ++c) ys[c] = 0.0f;
+            int e = 127;
+            float nb = 0.0f, tp = 0.0f;
+            float cf[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) cf[i] = 0.0f;
             const int ksteps = (g_end - g_begin) * 2;
-            int gcur = 0;           // this group's index in the slot sequence
-            float dm_next = 0.0f;   // this thread's d or m value of the next group
-            bool has_next = false;
+            int gcur = 0;
             for (int ks = 0; ks < ksteps && ok; ++ks, ++it) {
-                const int g = g_begin + (ks >> 1);  // global group index
                 const bool first_half = (ks & 1) == 0;
                 if (first_half) {
-                    // group set-up from the 8 block scales dx_0..dx_7 of this token:
+                    // ---- group set-up from this token's 8 block scales and sums ----
+                    const int slot = gi % kRing;
+                    if (!w4::mbar_wait(&scfull[slot], (uint32_t)(gi / kRing) & 1u, abort_flag,
+                                       p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t* src = sc + slot * Smem::kScSlotBytes;
+                    const float4 a0 = reinterpret_cast<const float4*>(src)[2 * row];
+                    const float4 a1 = reinterpret_cast<const float4*>(src)[2 * row + 1];
+                    const int4 s0 =
+                        reinterpret_cast<const int4*>(src + Smem::kScSlotBytes / 2)[2 * row];
+                    const int4 s1 =
+                        reinterpret_cast<const int4*>(src + Smem::kScSlotBytes / 2)[2 * row + 1];
+                    __syncwarp();
+                    if (lane == 0) w4::mbar_arrive(&scempty[slot]);
+                    gcur = gi;
+                    ++gi;
+                    const float dxg[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                    float tsum = 0.0f;  // sum_b dx_b S_b, fixed order
+                    tsum = fmaf(a0.x, (float)s0.x, tsum);
+                    tsum = fmaf(a0.y, (float)s0.y, tsum);
+                    tsum = fmaf(a0.z, (float)s0.z, tsum);
+                    tsum = fmaf(a0.w, (float)s0.w, tsum);
+                    tsum = fmaf(a1.x, (float)s1.x, tsum);
+                    tsum = fmaf(a1.y, (float)s1.y, tsum);
+                    tsum = fmaf(a1.z, (float)s1.z, tsum);
+                    tsum = fmaf(a1.w, (float)s1.w, tsum);
+                    float dmax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) dmax = fmaxf(dmax, dxg[i]);
+                    // e_want puts dmax * 2^e_want in [2^40, 2^41); a group whose
+                    // scales outgrow the token's current e by 2^24 or more moves
+                    // e down and rescales the partial output (e starts at 127)
+                    const int ex = (int)((__float_as_uint(dmax) >> 23) & 0xFFu);
+                    int e_want = 167 - ex;
+                    e_want = e_want < 22 ? 22 : (e_want > 127 ? 127 : e_want);
+                    if (e_want + 24 <= e) {
+                        const float r = pow2f(e_want - e);
+#pragma unroll
+                        for (int c = 0; c < kEpiCols; ++c) ys[c] *= r;
+                        e = e_want;
+                    }
+                    const float pe = pow2f(e);
                     // buffer r holds V_r = 2^17 + P_r after block r and
                     // V_{r+4} = 2^17 + P_r + P_{r+4} after block r + 4, so
                     //   sum_b dx_b P_b = sum_{r<4} (dx_r - dx_{r+4}) V_r + dx_{r+4} V_{r+4}
                     //                    - 2^17 sum_{r<4} dx_r
-                    float dxg[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) dxg[i] = 0.0f;
-                    tmin = 0.0f;
-                    float4 sa4[2];
-                    int4 ss4[2];
-                    {
-                        // this token's 8 scales and sums, brought in by TMA (zero past M)
-                        const int slot = gi & 1;
-                        if (!w4::mbar_wait(&scfull[slot], (uint32_t)(gi >> 1) & 1u, abort_flag,
-                                           p.err)) {
-                            ok = false;
-                            break;
-                        }
-                        const uint8_t* src = sc + slot * Smem::kScSlotBytes;
-                        sa4[0] = reinterpret_cast<const float4*>(src)[2 * row];
-                        sa4[1] = reinterpret_cast<const float4*>(src)[2 * row + 1];
-                        ss4[0] = reinterpret_cast<const int4*>(src + Smem::kScSlotBytes / 2)[2 * row];
-                        ss4[1] =
-                            reinterpret_cast<const int4*>(src + Smem::kScSlotBytes / 2)[2 * row + 1];
-                        __syncwarp();
-                        if (lane == 0) w4::mbar_arrive(&scempty[slot]);
-                    }
-                    gcur = gi;
-                    ++gi;
-                    // the next group's d or m, a whole group ahead of its use
-                    if (g + 1 < g_end) {
-                        has_next = true;
-                        dm_next = dm_value(n0, g + 1);
-                    } else if (u + (int)gridDim.x < p.units) {
-                        int tmi2, tni2, gb2, ge2;
-                        unit_of(u + gridDim.x, tmi2, tni2, gb2, ge2);
-                        has_next = true;
-                        dm_next = dm_value(tni2 * BN, gb2);
-                    } else {
-                        has_next = false;
-                    }
-                    {
-#pragma unroll
-                        for (int h4 = 0; h4 < 2; ++h4) {
-                            const float4 a = sa4[h4];
-                            const int4 sv = ss4[h4];
-                            dxg[4 * h4] = a.x;
-                            dxg[4 * h4 + 1] = a.y;
-                            dxg[4 * h4 + 2] = a.z;
-                            dxg[4 * h4 + 3] = a.w;
-                            tmin = fmaf(a.x, (float)sv.x, tmin);
-                            tmin = fmaf(a.y, (float)sv.y, tmin);
-                            tmin = fmaf(a.z, (float)sv.z, tmin);
-                            tmin = fmaf(a.w, (float)sv.w, tmin);
-                        }
-                    }
-                    float dmax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) dmax = fmaxf(dmax, dxg[i]);
-                    // e: dmax * 2^e in [2^40, 2^41), clamped to [22, 127]
-                    const int ex = (int)((__float_as_uint(dmax) >> 23) & 0xFFu);
-                    int e = 167 - ex;
-                    e = e < 22 ? 22 : (e > 127 ? 127 : e);
-                    const float pe = __uint_as_float((uint32_t)(e + 127) << 23);
-                    kpow = __uint_as_float((uint32_t)(149 - e + 127) << 23);
-                    neg_bias = -(float)(1 << kBiasLog2) * ((dxg[0] + dxg[1]) + (dxg[2] + dxg[3]));
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
                         cf[r] = (dxg[r] - dxg[r + 4]) * pe;
                         cf[r + 4] = dxg[r + 4] * pe;
                     }
+                    // -2^17 sum_{r<4} dx_r and sum_b dx_b S_b in units of 2^(e-149)
+                    nb = -(((dxg[0] + dxg[1]) + (dxg[2] + dxg[3])) * pe) * 0x1p-66f * 0x1p-66f;
+                    tp = (tsum * pe) * 0x1p-75f * 0x1p-74f;
                 }
+                // ---- the stage's 4 blocks as 8 chunks of 32 columns: load, wait,
+                // (release the buffer after its second half), 32 FMAs; the two
+                // epilogue warps of each SM sub-partition overlap one's loads with
+                // the other's FMAs ----
 #pragma unroll
-                for (int j = 0; j < NPAIR; ++j) {
-                    if (!ok) break;
-                    if (!w4::mbar_wait(&tfull[j], (uint32_t)it & 1u, abort_flag, p.err)) {
-                        ok = false;
-                        break;
+                for (int c = 0; c < 8; ++c) {
+                    const int q = c >> 1, h = c & 1;  // block (= buffer), 32-column half
+                    if (c == 0 || c == 4) {
+                        if (!w4::mbar_wait(&tfull[c >> 2], (uint32_t)it & 1u, abort_flag, p.err)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        // the second pair's commit covers all of the stage's MMAs:
+                        // its shared-memory operands can be refilled
+                        if (c == 4 && threadIdx.x == 128) w4::mbar_arrive(&sfree[it % STAGES]);
                     }
-                    tc_fence_after();
-                    // the stage's last pair has landed: its shared-memory operands are free
-                    if (j == NPAIR - 1 && threadIdx.x == 128) w4::mbar_arrive(&empty[it % STAGES]);
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        const int q = 2 * j + qq;  // block in the stage = buffer
-                        const float sc = first_half ? cf[q] : cf[q + 4];
-                        const uint32_t ta = tm_row + (uint32_t)(q * BN);
-                        // two 32-column halves; the pair is released once the
-                        // second block's words are in registers
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            uint32_t r[32];
-                            tmem_ld32(ta + 32 * hh, r);
-                            tmem_wait_ld();
-                            if (qq == 1 && hh == 1) {
-                                tc_fence_before();
-                                __syncwarp();
-                                if (lane == 0) w4::mbar_arrive(&tempty[j]);
+                    uint32_t rv[32];
+                    tmem_ld32(tm_row + (uint32_t)(q * BN + 32 * h), rv);
+                    tmem_wait_ld_regs(rv);
+                    if (h == 1) {
+                        // both halves of block q have been read: its buffer is free
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) w4::mbar_arrive(&tempty[q]);
+                    }
+                    if constexpr (kDump) {
+                        // block q (first stage) or q + 4 (second) of group g: the
+                        // running sum P_q, or P_q + P_{q+4}
+                        const int blk = (g_begin + (ks >> 1)) * 8 + (first_half ? q : q + 4);
+                        if (t_live) {
+                            for (int i = 0; i < 32; ++i) {
+                                const int n = n0 + cs * kEpiCols + 32 * h + i;
+                                if (n < p.N)
+                                    p.dump[((size_t)t * p.N + n) * (size_t)(p.K / 32) + blk] =
+                                        (int32_t)rv[i] - (1 << 17);
                             }
-#pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                acc[32 * hh + c] = fmaf(sc, __uint_as_float(r[c]), acc[32 * hh + c]);
                         }
                     }
+                    const float k = first_half ? cf[q] : cf[q + 4];
+                    if (first_half && q == 0) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            acc[32 * h + i] = fmaf(k, __uint_as_float(rv[i]), nb);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            acc[32 * h + i] = fmaf(k, __uint_as_float(rv[i]), acc[32 * h + i]);
+                    }
                 }
-                if (ok && !first_half) {
-                    // y += d * (acc * 2^(149-e) - 2^17 * sum_{r<4} dx_r) + m * sum dx S
-                    const int slot = gcur & 1;
-                    if (!w4::mbar_wait(&dmfull[slot], (uint32_t)(gcur >> 1) & 1u, abort_flag,
+                if (!ok) break;
+                if (!first_half) {
+                    // ---- group end: ys += d * acc + m * sum_b dx_b S_b ----
+                    const int slot = gcur % kRing;
+                    if (!w4::mbar_wait(&dmfull[slot], (uint32_t)(gcur / kRing) & 1u, abort_flag,
                                        p.err)) {
                         ok = false;
                         break;
                     }
-                    const float* ds = dm_s + slot * 2 * BN;
-                    const float4* dg = reinterpret_cast<const float4*>(ds + cs * kEpiCols);
-                    const float4* mg = reinterpret_cast<const float4*>(ds + BN + cs * kEpiCols);
+                    const float4* dg = reinterpret_cast<const float4*>(dm_s + slot * 2 * BN +
+                                                                       cs * kEpiCols);
+                    const float4* mg = dg + BN / 4;
 #pragma unroll
                     for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
                         const float4 dv = dg[c4], mv = mg[c4];
-                        const float dvv[4] = {dv.x, dv.y, dv.z, dv.w};
-                        const float mvv[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const int c = 4 * c4 + e4;
-                            const float av = fmaf(acc[c], kpow, neg_bias);
-                            yv[c] = fmaf(dvv[e4], av, fmaf(mvv[e4], tmin, yv[c]));
-                            acc[c] = 0.0f;
-                        }
+                        ys[4 * c4 + 0] = fmaf(dv.x, acc[4 * c4 + 0], fmaf(mv.x, tp, ys[4 * c4 + 0]));
+                        ys[4 * c4 + 1] = fmaf(dv.y, acc[4 * c4 + 1], fmaf(mv.y, tp, ys[4 * c4 + 1]));
+                        ys[4 * c4 + 2] = fmaf(dv.z, acc[4 * c4 + 2], fmaf(mv.z, tp, ys[4 * c4 + 2]));
+                        ys[4 * c4 + 3] = fmaf(dv.w, acc[4 * c4 + 3], fmaf(mv.w, tp, ys[4 * c4 + 3]));
                     }
                     __syncwarp();
                     if (lane == 0) w4::mbar_arrive(&dmfree[slot]);
-                    if (has_next) {
-                        // the other slot was last read at the previous group's end
-                        const int nslot = slot ^ 1;
-                        if (gcur >= 1 &&
-                            !w4::mbar_wait(&dmfree[nslot], (uint32_t)((gcur - 1) >> 1) & 1u,
-                                           abort_flag, p.err)) {
-                            ok = false;
-                            break;
-                        }
-                        dm_s[nslot * 2 * BN + et] = dm_next;
-                        __syncwarp();
-                        if (lane == 0) w4::mbar_arrive(&dmfull[nslot]);
-                    }
                 }
             }
+            // back to the output's own scale: y = ys * 2^(149 - e)
+            {
+                const float kpow = pow2f(149 - e);
+#pragma unroll
+                for (int c = 0; c < kEpiCols; ++c) ys[c] *= kpow;
+            }
             // ---- store: directly, or through the split-K workspace ----
-            const int nb = n0 + cs * kEpiCols;
+            const int nb0 = n0 + cs * kEpiCols;
             bool store = ok && t_live;
             if (p.splits > 1) {
                 // every epilogue thread reaches both barriers, aborted or not
@@ -643,8 +672,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    (size_t)cs * (kEpiCols / 4) * BM + row;
 #pragma unroll
                     for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
-                        mine[(size_t)c4 * BM] = make_float4(yv[4 * c4], yv[4 * c4 + 1],
-                                                            yv[4 * c4 + 2], yv[4 * c4 + 3]);
+                        mine[(size_t)c4 * BM] = make_float4(ys[4 * c4], ys[4 * c4 + 1],
+                                                            ys[4 * c4 + 2], ys[4 * c4 + 3]);
                 }
                 __threadfence();
                 asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -662,16 +691,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         reinterpret_cast<const float4*>(p.partials + (size_t)tile * p.splits * BM * BN) +
                         (size_t)cs * (kEpiCols / 4) * BM + row;
 #pragma unroll
-                    for (int c = 0; c < kEpiCols; ++c) yv[c] = 0.0f;
+                    for (int c = 0; c < kEpiCols; ++c) ys[c] = 0.0f;
                     for (int q = 0; q < p.splits; ++q) {
                         const float4* src = base + (size_t)q * (BM * BN / 4);
 #pragma unroll
                         for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
                             const float4 v = __ldcg(src + (size_t)c4 * BM);
-                            yv[4 * c4] += v.x;
-                            yv[4 * c4 + 1] += v.y;
-                            yv[4 * c4 + 2] += v.z;
-                            yv[4 * c4 + 3] += v.w;
+                            ys[4 * c4] += v.x;
+                            ys[4 * c4 + 1] += v.y;
+                            ys[4 * c4 + 2] += v.z;
+                            ys[4 * c4 + 3] += v.w;
                         }
                     }
                     if (threadIdx.x == 128) p.counters[tile] = 0;  // ready for the next call
@@ -680,36 +709,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (store) {
                 if (p.out_f32) {
                     float* yr = reinterpret_cast<float*>(p.y) + (size_t)t * p.N;
-                    if (nb + kEpiCols <= p.N && (p.N & 3) == 0) {
+                    if (nb0 + kEpiCols <= p.N && (p.N & 3) == 0) {
 #pragma unroll
                         for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
-                            *reinterpret_cast<float4*>(yr + nb + 4 * c4) = make_float4(
-                                yv[4 * c4], yv[4 * c4 + 1], yv[4 * c4 + 2], yv[4 * c4 + 3]);
+                            *reinterpret_cast<float4*>(yr + nb0 + 4 * c4) = make_float4(
+                                ys[4 * c4], ys[4 * c4 + 1], ys[4 * c4 + 2], ys[4 * c4 + 3]);
                     } else {
 #pragma unroll
                         for (int c = 0; c < kEpiCols; ++c)
-                            if (nb + c < p.N) yr[nb + c] = yv[c];
+                            if (nb0 + c < p.N) yr[nb0 + c] = ys[c];
                     }
                 } else {
                     __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)t * p.N;
-                    if (nb + kEpiCols <= p.N && (p.N & 7) == 0) {
+                    if (nb0 + kEpiCols <= p.N && (p.N & 7) == 0) {
 #pragma unroll
                         for (int c8 = 0; c8 < kEpiCols / 8; ++c8) {
                             uint4 v;
-                            __nv_bfloat162 h0 = __floats2bfloat162_rn(yv[8 * c8 + 0], yv[8 * c8 + 1]);
-                            __nv_bfloat162 h1 = __floats2bfloat162_rn(yv[8 * c8 + 2], yv[8 * c8 + 3]);
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(yv[8 * c8 + 4], yv[8 * c8 + 5]);
-                            __nv_bfloat162 h3 = __floats2bfloat162_rn(yv[8 * c8 + 6], yv[8 * c8 + 7]);
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(ys[8 * c8 + 0], ys[8 * c8 + 1]);
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(ys[8 * c8 + 2], ys[8 * c8 + 3]);
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(ys[8 * c8 + 4], ys[8 * c8 + 5]);
+                            __nv_bfloat162 h3 = __floats2bfloat162_rn(ys[8 * c8 + 6], ys[8 * c8 + 7]);
                             v.x = *reinterpret_cast<uint32_t*>(&h0);
                             v.y = *reinterpret_cast<uint32_t*>(&h1);
                             v.z = *reinterpret_cast<uint32_t*>(&h2);
                             v.w = *reinterpret_cast<uint32_t*>(&h3);
-                            *reinterpret_cast<uint4*>(yr + nb + 8 * c8) = v;
+                            *reinterpret_cast<uint4*>(yr + nb0 + 8 * c8) = v;
                         }
                     } else {
 #pragma unroll
                         for (int c = 0; c < kEpiCols; ++c)
-                            if (nb + c < p.N) yr[nb + c] = __float2bfloat16_rn(yv[c]);
+                            if (nb0 + c < p.N) yr[nb0 + c] = __float2bfloat16_rn(ys[c]);
                     }
                 }
             }
@@ -845,13 +874,14 @@ int validate_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
-             int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
-             void* y, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
-    int rc = validate_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype);
-    if (rc != W4_OK) return rc;
+// Launch of the product after validate_mmq: tensor maps, split-K workspace,
+// one persistent CTA per SM.  dump != nullptr selects the test instantiation.
+int launch_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
+               int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
+               void* y, int out_dtype, void* workspace, size_t ws_bytes, int32_t* dump,
+               void* stream) {
     int* err = w4::device_error_word();
     if (!err) return W4_ERR_CUDA;
     const int splits = pick_splits(M, N, K, w4::sm_count());
@@ -877,15 +907,20 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
         !make_map_4b(&ms, bsum, CU_TENSOR_MAP_DATA_TYPE_INT32, (uint64_t)K / 32, (uint64_t)M, 8,
                      BM))
         return W4_ERR_CUDA;
-    static thread_local int attr_dev = -1;
+    static thread_local int attr_dev[2] = {-1, -1};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return w4::cuda_fail(e);
-    if (attr_dev != dev) {
-        e = cudaFuncSetAttribute(w4a8_mmq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)Smem::total);
+    const int which = dump ? 1 : 0;
+    if (attr_dev[which] != dev) {
+        e = dump ? cudaFuncSetAttribute(w4a8_mmq_kernel<true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)Smem::total)
+                 : cudaFuncSetAttribute(w4a8_mmq_kernel<false>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)Smem::total);
         if (e != cudaSuccess) return w4::cuda_fail(e);
-        attr_dev = dev;
+        attr_dev[which] = dev;
     }
     Params prm;
     prm.d = reinterpret_cast<const __half*>(d_f16);
@@ -901,6 +936,7 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     prm.splits = splits;
     prm.counters = nullptr;
     prm.partials = nullptr;
+    prm.dump = dump;
     if (splits > 1) {
         prm.counters = static_cast<int*>(workspace);
         prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
@@ -911,7 +947,59 @@ int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
     prm.tiles_n = (int)((N + BN - 1) / BN);
     prm.units = (int)(tiles * splits);
     const int grid = prm.units < w4::sm_count() ? prm.units : w4::sm_count();
-    w4a8_mmq_kernel<<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, mdx, ms, prm);
+    if (dump)
+        w4a8_mmq_kernel<true><<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, mdx, ms, prm);
+    else
+        w4a8_mmq_kernel<false><<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, mdx, ms, prm);
+    return w4::launch_status();
+}
+
+
+// The dump holds, per (token, row, group), running sums R_r = P_r and
+// R_{r+4} = P_r + P_{r+4} (r < 4) as read from TMEM; this turns the second
+// half into block products P_{r+4} = R_{r+4} - R_r.
+__global__ void blockdots_from_running_sums(int32_t* __restrict__ P, int64_t rows, int G) {
+    const int64_t total = rows * (int64_t)G * 4;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t rg = i >> 2;  // (token, row, group)
+        const int r = (int)(i & 3);
+        int32_t* grp = P + rg * 8;
+        grp[r + 4] -= grp[r];
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int w4a8_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16, int64_t N,
+             int64_t K, const int8_t* qa, const float* dx, const int32_t* bsum, int64_t M,
+             void* y, int out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+    int rc = validate_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype);
+    if (rc != W4_OK) return rc;
+    return launch_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype, workspace,
+                      ws_bytes, nullptr, stream);
+}
+
+int w4a8_mmq_blockdots(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f16,
+                       int64_t N, int64_t K, const int8_t* qa, const float* dx,
+                       const int32_t* bsum, int64_t M, void* y, int out_dtype,
+                       int32_t* blockdots, size_t bd_bytes, void* workspace, size_t ws_bytes,
+                       void* stream) {
+    int rc = validate_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype);
+    if (rc != W4_OK) return rc;
+    if (!blockdots) return W4_ERR_NULL;
+    if (!w4::aligned16(blockdots)) return W4_ERR_ALIGN;
+    if (bd_bytes < (size_t)M * (size_t)N * (size_t)(K / 32) * 4) return W4_ERR_WORKSPACE;
+    rc = launch_mmq(codes, d_f16, m_f16, N, K, qa, dx, bsum, M, y, out_dtype, workspace,
+                    ws_bytes, blockdots, stream);
+    if (rc != W4_OK) return rc;
+    const int64_t total = M * N * (K / 256) * 4;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)w4::sm_count() * 8) blocks = (int64_t)w4::sm_count() * 8;
+    blockdots_from_running_sums<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(
+        blockdots, M * N, (int)(K / 256));
     return w4::launch_status();
 }
 
