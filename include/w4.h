@@ -112,12 +112,15 @@ int w4_pack_g32(const float *w, int64_t N, int64_t K, uint8_t *codes,
                 uint16_t *d_f16, uint16_t *m_f16, void *stream);
 
 /* Pack one-code-per-byte q [N][K] (values 0..15; higher bits are ignored)
- * into codes [N][K/2] with the nibble order above.  K % 2 == 0 and
- * (N*K) % 32 == 0. */
+ * into codes [N][K/2] with the nibble order above: the 128-byte packed code
+ * block of each group of the HFQ4-G256 format (the hipfire MMQ article's
+ * weight format; the nibble order is the reading stated at the top of this
+ * file).  K % 2 == 0 and (N*K) % 32 == 0. */
 int w4_pack_codes(const uint8_t *q, int64_t N, int64_t K, uint8_t *codes,
                   void *stream);
 
-/* Inverse of w4_pack_codes: codes [N][K/2] -> q [N][K], one code per byte.
+/* Inverse of w4_pack_codes: codes [N][K/2] -> q [N][K], one code per byte
+ * (the 4-bit codes q in [0,15] of the HFQ4-G256 format, hipfire MMQ article).
  * K % 2 == 0 and (N*K) % 32 == 0. */
 int w4_unpack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *q,
               void *stream);
@@ -128,7 +131,12 @@ int w4_unpack(const uint8_t *codes, int64_t N, int64_t K, uint8_t *q,
  *                     + m[n][g] * sum_{k in g} x[t][k] )
  * for t < M, n < N, accumulated in fp32.
  * codes/d/m: the format planes of W[N][K]; x: bf16 [M][K]; y: [M][N] of
- * out_dtype.  1 <= M <= 8, N >= 1, K >= 256, K % 256 == 0. */
+ * out_dtype.  1 <= M <= 8, N >= 1, 256 <= K <= 65536, K % 256 == 0; larger
+ * sizes give W4_ERR_SHAPE.  Each launch stages its tokens' activations in
+ * shared memory (72 bytes per token and 32 k in this bf16 form, 40 bytes in
+ * the int8 forms, at most 200 KB): when M tokens do not fit (e.g. M = 8 at
+ * K = 12288) they are processed in passes of as many tokens as fit, each pass
+ * streaming the weights again. */
 int w4_gemv(const uint8_t *codes, const uint16_t *d_f16,
             const uint16_t *m_f16, int64_t N, int64_t K,
             const uint16_t *x_bf16, int M, void *y, int out_dtype,
@@ -138,8 +146,9 @@ int w4_gemv(const uint8_t *codes, const uint16_t *d_f16,
  *   y[t][n] = sum_g ( d[n][g] * sum_{k in g} q[n][k] * x[t][k]
  *                     + m[n][g] * sum_{k in g} x[t][k] ),  groups of 32,
  * accumulated in fp32.  codes [N][K/2], d and m [N][K/32] from w4_pack_g32;
- * x: bf16 [M][K]; y: [M][N] of out_dtype.  1 <= M <= 8, N >= 1, K >= 32,
- * K % 32 == 0.  Same validation and errors as w4_gemv. */
+ * x: bf16 [M][K]; y: [M][N] of out_dtype.  1 <= M <= 8, N >= 1,
+ * 32 <= K <= 65536, K % 32 == 0.  Same validation, errors and token passes
+ * as w4_gemv. */
 int w4_gemv_g32(const uint8_t *codes, const uint16_t *d_f16,
                 const uint16_t *m_f16, int64_t N, int64_t K,
                 const uint16_t *x_bf16, int M, void *y, int out_dtype,
@@ -156,8 +165,9 @@ int w4_gemv_g32(const uint8_t *codes, const uint16_t *d_f16,
  *                        + m[n][g] * sum_{b in g} dx[t][b] * S[t][b] )
  * scales applied in fp32.  codes/d/m: W[N][K] planes; qa int8 [M][K], dx fp32
  * [M][K/32], bsum int32 [M][K/32]: the output of q8_quantize_act; y: [M][N]
- * of out_dtype.  1 <= M <= 8, N >= 1, K >= 256, K % 256 == 0; every pointer
- * 16-byte aligned.  Same validation and errors as w4_gemv. */
+ * of out_dtype.  1 <= M <= 8, N >= 1, 256 <= K <= 65536, K % 256 == 0;
+ * every pointer 16-byte aligned.  Same validation, errors and token passes as
+ * w4_gemv. */
 int w4a8_gemv(const uint8_t *codes, const uint16_t *d_f16,
               const uint16_t *m_f16, int64_t N, int64_t K, const int8_t *qa,
               const float *dx, const int32_t *bsum, int M, void *y,
@@ -186,7 +196,11 @@ int q8_quantize_act(const uint16_t *x_bf16, int64_t M, int64_t K, int8_t *qa,
                     float *dx, int32_t *bsum, void *stream);
 
 /* Bytes of device workspace w4a8_mmq needs for this shape (0 means none; the
- * workspace pointer may then be NULL). */
+ * workspace pointer may then be NULL).  The workspace holds the fp32 partial
+ * output tiles of a split over K, used when the output tiles alone do not fill
+ * the GPU (the tiled int8 matrix-matrix product of the hipfire MMQ article
+ * runs here as 128x128 tiles; the split is this library's, not the
+ * article's): int32 arrival counters, then [tiles][splits][128][128] fp32. */
 size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* W4A8 prefill product on int8 tensor cores (the article's MMQ path: int8
@@ -261,6 +275,21 @@ int w4a8_mmq_blockdots(const uint8_t *codes, const uint16_t *d_f16,
                        int64_t M, void *y, int out_dtype, int32_t *blockdots,
                        size_t bd_bytes, void *workspace, size_t ws_bytes,
                        void *stream);
+
+/* w4a8_gemv that also returns the exact integer block products its integer
+ * core formed:
+ *   blockdots[t][n][b] = P[t][n][b] = sum_{k in block b} q[n][k] * qa[t][k]
+ * (int32 [M][N][K/32], row-major; bd_bytes >= M*N*(K/32)*4, else
+ * W4_ERR_WORKSPACE), stored by the test instantiation of the same kernels,
+ * with the same dispatch, that w4a8_gemv runs, so that the decode path's
+ * integer core can be compared with the CPU bit for bit (the keep-quant
+ * integer core of the GFX1100-TG150 spec, "Design").  y and every other
+ * argument and error are those of w4a8_gemv.  For tests. */
+int w4a8_gemv_blockdots(const uint8_t *codes, const uint16_t *d_f16,
+                        const uint16_t *m_f16, int64_t N, int64_t K,
+                        const int8_t *qa, const float *dx, const int32_t *bsum,
+                        int M, void *y, int out_dtype, int32_t *blockdots,
+                        size_t bd_bytes, void *stream);
 
 /* Runs the bounded-wait routine that every pipelined kernel of this library
  * uses, on a wait that can never complete: one thread waits on an mbarrier

@@ -138,3 +138,23 @@ def test_rejects_bad_arguments(torch, w4):
     with pytest.raises(w4.W4Error):
         w4.w4_gemv(codes, d, d, x, y=y_mis)
     w4.w4_check_device_error()
+
+
+@pytest.mark.parametrize("M,K", [(8, 12288), (5, 16384), (8, 20480), (1, 65536)])
+def test_large_k_every_m(torch, w4, orc, M, K):
+    # K where M tokens' staged activations exceed one launch's shared memory:
+    # the tokens go in passes (the 9B-class down-projection K = 12288 at the
+    # M = 8 verify batch among them); every output against the oracle
+    N = 300
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=M + K)
+    x = synth.activations(M, K, seed=K + 7 * M)
+    _both(torch, w4, orc, codes, d, m, x, what=f"M{M} K{K}")
+
+
+def test_k_above_the_limit_is_refused(torch, w4):
+    codes = torch.zeros((16, 65792 // 2), dtype=torch.uint8, device="cuda")
+    d = torch.zeros((16, 65792 // 256), dtype=torch.float16, device="cuda")
+    x = torch.zeros((1, 65792), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(w4.W4Error):
+        w4.w4_gemv(codes, d, d, x)
+

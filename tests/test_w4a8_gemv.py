@@ -176,3 +176,28 @@ def test_fused_quantiser_is_bit_identical(torch, w4, orc, M, N, K):
     ref = np.concatenate([orc.mmq(codes, d, m, qa_o, dx_o, S_o, rows=(int(r), int(r) + 1))
                           for r in rows], axis=1)
     parity.assert_f32_gate(fused.cpu().numpy()[:, rows], ref, f"fused M{M} {N}x{K}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 6144, 2560), (3, 300, 768), (8, 260, 2560),
+                                   (4, 2560, 9728), (8, 200, 12288), (2, 20000, 2560)])
+def test_integer_block_products_bit_exact(torch, w4, orc, M, N, K):
+    # The exact int32 block products of the integer core, stored by the test
+    # instantiation of the same kernels and dispatch (ring kernel for the small
+    # streams, row kernel for the 25.6 MB one; token passes at M = 8, K = 12288),
+    # equal the oracle's int64 products element for element; y of the same call
+    # is bitwise that of w4a8_gemv.
+    codes, d, m = synth.quantized_weights_direct(N, K, seed=3 * M + N + K)
+    qa, dx, S = orc.q8_quantize(synth.outlier_activations(M, K, seed=M + N + 5 * K))
+    dev = (torch.from_numpy(codes).cuda(), _dev_u16(torch, d, torch.float16),
+           _dev_u16(torch, m, torch.float16), torch.from_numpy(qa).cuda(),
+           torch.from_numpy(dx).cuda(), torch.from_numpy(S).cuda())
+    y, P = w4.w4a8_gemv_blockdots(*dev, out_dtype=torch.float32)
+    y2 = w4.w4a8_gemv(*dev, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    want = orc.mmq_blockdots(codes, qa)
+    got = P.cpu().numpy().astype(np.int64)
+    bad = int((got != want).sum())
+    assert bad == 0, f"{bad} of {want.size} block products differ"
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32))
+    parity.assert_f32_gate(y.cpu().numpy(), orc.mmq(codes, d, m, qa, dx, S), f"M{M} N{N} K{K}")
+

@@ -19,6 +19,7 @@ Entry points (same names as the C ABI):
     w4a8_mmq(codes, d, m, qa, dx, bsum, out_dtype) -> y
     w4a8_mmq_static(codes, d, m, qa, dx, bsum, out_dtype) -> y   (no workspace)
     w4a8_mmq_blockdots(codes, d, m, qa, dx, bsum, out_dtype) -> y, P   (test: int32 block products)
+    w4a8_gemv_blockdots(codes, d, m, qa, dx, bsum, out_dtype) -> y, P  (test: int32 block products)
     w4a8_mmq_workspace_size(M, N, K)
     w4_check_device_error()
 """
@@ -31,7 +32,7 @@ __all__ = [
     "w4_gemv", "w4_gemv_g32", "w4a8_gemv",
     "w4a8_gemv_bf16",
     "q8_quantize_act", "w4a8_mmq", "w4a8_mmq_static", "w4a8_mmq_workspace_size",
-    "w4a8_mmq_blockdots",
+    "w4a8_mmq_blockdots", "w4a8_gemv_blockdots",
     "w4_check_device_error",
     "w4_abi_version", "lib",
 ]
@@ -374,5 +375,21 @@ def w4a8_mmq_blockdots(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, stream
                                      _ptr(bsum), M, _ptr(y), oc, _ptr(P),
                                      P.numel() * 4, _ptr(ws) if ws is not None else None,
                                      ws_need, _stream(stream)), "w4a8_mmq_blockdots")
+    return y, P
+
+
+def w4a8_gemv_blockdots(codes, d, m, qa, dx, bsum, out_dtype=None, y=None, stream=None):
+    """w4a8_gemv (M <= 8) that also returns the exact int32 block products
+    P[M, N, K/32] its integer core formed (for tests).  Returns (y, P)."""
+    torch = _torch()
+    M, K = _int8_acts(qa, dx, bsum)
+    N = _weights(codes, d, m, K)
+    oc = _out_code(out_dtype, y)
+    y = _output(y, M, N, oc, qa)
+    _on_device(codes=codes, d=d, m=m, qa=qa, dx=dx, bsum=bsum, y=y)
+    P = torch.empty((M, N, K // BLOCK), dtype=torch.int32, device=qa.device)
+    _check(load().w4a8_gemv_blockdots(_ptr(codes), _ptr(d), _ptr(m), N, K, _ptr(qa), _ptr(dx),
+                                      _ptr(bsum), M, _ptr(y), oc, _ptr(P), P.numel() * 4,
+                                      _stream(stream)), "w4a8_gemv_blockdots")
     return y, P
 

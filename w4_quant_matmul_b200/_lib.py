@@ -46,6 +46,8 @@ SIGNATURES = {
                  _INT),
     "w4a8_mmq_static": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P], _INT),
     "w4_test_wait_expiry": ([ctypes.c_uint64, _P], _INT),
+    "w4a8_gemv_blockdots": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _INT, _P, _INT, _P,
+                             ctypes.c_size_t, _P], _INT),
     "w4a8_mmq_blockdots": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _I64, _P, _INT, _P,
                             ctypes.c_size_t, _P, ctypes.c_size_t, _P], _INT),
 }

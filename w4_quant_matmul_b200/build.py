@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libw4.so")
-SOURCES = ["abi.cu", "pack.cu", "quant.cu", "gemv.cu", "mmq.cu"]
+SOURCES = ["abi.cu", "pack.cu", "quant.cu", "gemv.cu", "gemv_blockdots.cu", "mmq.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # No --use_fast_math / -ftz=true / -prec-div=false: the W4A8 product's epilogue
 # multiplies exact integer products held as fp32 denormals, which a
