@@ -94,6 +94,13 @@ def load_peaks() -> dict:
             "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def l2_flush(buf) -> None:
+    """Evict L2 (126 MB) by reading a 256 MB buffer.  A read leaves L2 full of
+    clean lines; a write would leave dirty lines whose write-back the next,
+    timed kernel would pay for."""
+    buf.max()
+
+
 def source_hash(*files: str) -> str:
     h = hashlib.sha256()
     for f in files:
@@ -121,63 +128,108 @@ def load_traffic(kernel_file: str, key: str):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled DURING a region.
+
+    NVML is polled from a thread every `interval_s` (0.5 ms by default, so that
+    even a region of a few milliseconds gets samples); if NVML is missing,
+    `nvidia-smi -lms 100` is read instead.  Reasons reported: hw_slowdown,
+    hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_s: float = 0.0005):
         self.gpu = gpu_index
+        self.interval = interval_s
+        self.samples: list[tuple[float, float, set]] = []  # (sm MHz, max MHz, reasons)
         self.proc = None
-        self.lines: list[str] = []
         self.thread = None
+        self.stop = threading.Event()
+        self.nvml = None
 
     def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                  pynvml.NVML_CLOCK_SM))
+            self.bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                         "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                         "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                         "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.sample_once()
+            self.thread.start()
+            return self
+        except Exception:  # no NVML: fall back to nvidia-smi
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except (OSError, ValueError):
             self.proc = None
         return self
 
-    def _read(self):
+    def sample_once(self):
+        pynvml = self.nvml
+        sm = float(pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        mask = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+        self.samples.append((sm, self.max_mhz, {n for n, b in self.bits.items() if mask & b}))
+
+    def _poll_nvml(self):
+        while not self.stop.is_set():
+            try:
+                self.sample_once()
+            except Exception:
+                return
+            time.sleep(self.interval)
+
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            self.samples.append((sm, smax, {n for n, v in zip(self.NAMES, parts[5:9])
+                                            if v.lower() == "active"}))
 
     def __exit__(self, *exc):
+        self.stop.set()
+        if self.nvml is not None:
+            try:
+                self.sample_once()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            if self.thread:
-                self.thread.join(timeout=2)
+        if self.thread:
+            self.thread.join(timeout=2)
 
     def summary(self) -> dict:
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = set()
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples),
+                "sm_max_mhz": max(m for _, m, _ in self.samples),
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "source": "nvml" if self.nvml is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -305,7 +357,7 @@ def time_gemv_sweep(torch, w4, wl, M, steps, warmup, stream):
     return elapsed, per, steps * len(SHAPES)
 
 
-def time_w4a8_gemv(torch, w4, wl, M, steps, stream, fused=False):
+def time_w4a8_gemv(torch, w4, wl, M, steps, stream, fused=False, pair=False):
     """Keep-quant decode GEMV (int8 activation blocks from q8_quantize_act,
     quantised once outside the timed launches): per-shape mean ms, each launch
     its own CUDA graph between events, shapes in sweep order so the lm_head
@@ -321,6 +373,8 @@ def time_w4a8_gemv(torch, w4, wl, M, steps, stream, fused=False):
                               stream=stream)
             return
         qa, dx, S = acts[s]
+        if pair:  # the two-step path it replaces: quantiser, then the GEMV
+            w4.q8_quantize_act(xs[s], qa, dx, S, stream=stream)
         w4.w4a8_gemv(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=ys[s], stream=stream)
 
     graphs = [[_capture(torch, stream, lambda c=c, s=s: run(c, s)) for s in range(len(SHAPES))]
@@ -432,7 +486,7 @@ def _time_mmq(torch, w4, dev, stream, reps):
     out = []
     g = torch.Generator(device=dev)
     g.manual_seed(11)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
     for si, (N, K) in enumerate(synth.MMQ_SHAPES):
         w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
         codes, d, m = w4.w4_pack(w)
@@ -448,7 +502,7 @@ def _time_mmq(torch, w4, dev, stream, reps):
             tq, tm = [], []
             for _ in range(reps):
                 with torch.cuda.stream(stream):
-                    flush.zero_()  # L2 flush, ordered before the timed launches
+                    l2_flush(flush)  # ordered before the timed launches
                 e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
                 e0.record(stream)
                 w4.q8_quantize_act(x, qa, dx, S, stream=stream)
@@ -460,11 +514,43 @@ def _time_mmq(torch, w4, dev, stream, reps):
                 tm.append(e1.elapsed_time(e2) / 1e3)
             t_mmq = statistics.median(tm)
             t_q = statistics.median(tq)
+            # the prefill pair (quantiser -> product) as one CUDA graph, the
+            # product launched programmatically dependent on the quantiser,
+            # against the two launches as separate graphs back to back
+            ws_need = w4.w4a8_mmq_workspace_size(M, N, K)
+            ws = torch.empty(max(ws_need, 16), dtype=torch.uint8, device=dev)
+
+            def quant():
+                w4.q8_quantize_act(x, qa, dx, S, stream=stream)
+
+            def prod():
+                w4.w4a8_mmq(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y,
+                            workspace=ws if ws_need else None, stream=stream)
+
+            g_pair = _capture(torch, stream, lambda: (quant(), prod()))
+            g_q = _capture(torch, stream, quant)
+            g_m = _capture(torch, stream, prod)
+            tp, ts = [], []
+            for _ in range(reps):
+                for graphs, acc in (((g_pair,), tp), ((g_q, g_m), ts)):
+                    with torch.cuda.stream(stream):
+                        l2_flush(flush)
+                    e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+                    e0.record(stream)
+                    for gr in graphs:
+                        gr.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    acc.append(e0.elapsed_time(e1) / 1e3)
+            del g_pair, g_q, g_m
+            t_pair, t_sep = statistics.median(tp), statistics.median(ts)
             out.append({"M": M, "N": N, "K": K, "mmq_us": t_mmq * 1e6,
                         "tops": mmq_ops(M, N, K) / t_mmq / 1e12,
                         "quant_us": t_q * 1e6, "quant_gbs": quant_bytes(M, K) / t_q / 1e9,
-                        "mmq_min_us": min(tm) * 1e6, "mmq_max_us": max(tm) * 1e6})
-            del x, qa, dx, S, y
+                        "mmq_min_us": min(tm) * 1e6, "mmq_max_us": max(tm) * 1e6,
+                        "pair_graph_us": round(t_pair * 1e6, 2),
+                        "separate_graphs_us": round(t_sep * 1e6, 2)})
+            del x, qa, dx, S, y, ws
     del flush
     return out
 
@@ -528,6 +614,10 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
     world, rank, local = dist_env()
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: for N > 1 launch one "
+                         "process per GPU (python -m torch.distributed.run --nproc-per-node N "
+                         "bench.py --gpus N ...)")
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     if world > 1:
@@ -587,7 +677,10 @@ def run_ours(args):
                   "gbs": round(gemv_bytes(n, k, 1) / (ms / 1e3) / 1e9, 1)}
                  for (n, k), ms in zip(SHAPES, per_shape_ms)]
     extras["gemv_m1"] = per_shape
+    section_clocks = {}
     if not args.quick:
+        sec = ClockSampler(local, interval_s=0.005)
+        sec.__enter__()
         for M in synth.SMALL_BATCH:
             e, per, _ = time_gemv_sweep(torch, w4, wl, M, max(3, args.steps // 2), 2, stream)
             extras[f"gemv_m{M}"] = [{"N": n, "K": k, "us": round(ms * 1e3, 2),
@@ -604,14 +697,20 @@ def run_ours(args):
             # the same product from bf16 x, quantiser folded in (algorithmic
             # bytes: the bf16 GEMV's)
             per = time_w4a8_gemv(torch, w4, wl, M, max(3, args.steps // 2), stream, fused=True)
+            two = time_w4a8_gemv(torch, w4, wl, M, max(3, args.steps // 2), stream, pair=True)
             extras[f"w4a8_gemv_bf16_m{M}"] = [
                 {"N": n, "K": k, "us": round(ms * 1e3, 2),
                  "gbs": round(gemv_bytes(n, k, M) / (ms / 1e3) / 1e9, 1),
-                 "tok_per_s": round(M / (ms / 1e3), 1)}
-                for (n, k), ms in zip(SHAPES, per)]
+                 "tok_per_s": round(M / (ms / 1e3), 1),
+                 "two_step_us": round(ms2 * 1e3, 2)}
+                for (n, k), ms, ms2 in zip(SHAPES, per, two)]
+        sec.__exit__(None, None, None)
+        section_clocks["decode_extras"] = sec.summary()
         del wl
         torch.cuda.empty_cache()
-        mmq = time_mmq(torch, w4, dev, stream)
+        with ClockSampler(local, interval_s=0.005) as sec:
+            mmq = time_mmq(torch, w4, dev, stream)
+        section_clocks["mmq"] = sec.summary()
         int8_peak = peaks["bf16_tflops"] * INT8_OVER_BF16
         for r in mmq:
             r["frac_int8_peak"] = round(r["tops"] / int8_peak, 4)
@@ -620,8 +719,12 @@ def run_ours(args):
         extras["int8_peak_tops"] = {"value": int8_peak,
                                     "how": f"{peaks['source']} bf16 burst x {INT8_OVER_BF16}"}
         torch.cuda.empty_cache()
-        extras["chain"] = time_chain(torch, w4, dev, stream)
+        with ClockSampler(local, interval_s=0.005) as sec:
+            extras["chain"] = time_chain(torch, w4, dev, stream)
+        section_clocks["chain"] = sec.summary()
         extras["chain"]["frac_hbm"] = round(extras["chain"]["gbs"] / peaks["hbm_gbs"], 4)
+    if section_clocks:
+        extras["clocks_by_section"] = section_clocks
     w4.w4_check_device_error()
 
     cpu = None
@@ -665,24 +768,73 @@ def _oracle_sample(rows_per_shape: int):
     return o, sample
 
 
-def cpu_baseline(seconds: float = 15.0, rows_per_shape: int = 2048) -> dict:
-    """The oracle GEMV (fp64, OpenMP over rows) on a bounded sample of the
-    batch-1 sweep, timed on this host's cores."""
-    o, sample = _oracle_sample(rows_per_shape)
-    nbytes = sum(gemv_bytes(n, K, 1) for (_, _, _, _, n, K) in sample)
+def _cpu_model() -> str:
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name:"):
+                return line.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return "unknown"
+
+
+def _timed_passes(fn, seconds: float):
+    """Run fn() until `seconds` have passed (at least once); (passes, s)."""
     t0 = time.perf_counter()
     reps = 0
     while True:
-        for codes, d, m, x, n, K in sample:
-            o.gemv(codes, d, m, x)
+        fn()
         reps += 1
-        if time.perf_counter() - t0 >= seconds:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": round(nbytes * reps / dt / 1e9, 3), "unit": "GB/s",
-            "cores": o.num_threads(), "kind": "oracle",
-            "sample": f"{rows_per_shape} rows of each of the 5 batch-1 shapes (M=1), "
-                      f"{reps} passes, {dt:.1f} s"}
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            return reps, dt
+
+
+def cpu_baseline(seconds: float = 15.0, rows_per_shape: int = 2048) -> dict:
+    """The oracle (fp64 / int64, OpenMP over output rows) timed on this host's
+    cores, on bounded samples of the configurations, on one core and on all
+    cores: the batch-1 sweep (`value`, all cores, GB/s of the sampled rows),
+    the tiny case in full, the W4A8 product on a 256-token x 256-row slice of
+    the prefill shape, and the per-token chain as the batch-1 rate applied to
+    the chain's 2.078 GB."""
+    import oracle
+    o, sample = _oracle_sample(rows_per_shape)
+    all_cores = len(os.sched_getaffinity(0))
+    nbytes = sum(gemv_bytes(n, K, 1) for (_, _, _, _, n, K) in sample)
+    tiny = synth.tiny(0)
+    N, K = synth.MMQ_SHAPES[0]
+    w = synth.dense_weights(256, K, synth.weight_seed(synth.CONFIG_MMQ, 0))
+    mc, md, mm = o.w4_pack(w)
+    qa, dx, S = o.q8_quantize(synth.outlier_activations(256, K, synth.act_seed(synth.CONFIG_MMQ, 0)))
+    chain_bytes = (synth.CHAIN_LAYERS * sum(gemv_bytes(n, k, 1) for n, k in synth.LAYER_SHAPES)
+                   + gemv_bytes(*synth.LM_HEAD, 1))
+    runs = {}
+    budget = {1: 0.3 * seconds, all_cores: 0.7 * seconds}
+    try:
+        for cores in sorted(set([1, all_cores])):
+            o.set_num_threads(cores)
+            b = budget.get(cores, 0.5 * seconds)
+            reps, dt = _timed_passes(lambda: [o.gemv(c, d, m, x) for c, d, m, x, n, k in sample],
+                                     0.6 * b)
+            gbs = nbytes * reps / dt / 1e9
+            treps, tdt = _timed_passes(lambda: o.gemv(*tiny), 0.05 * b)
+            mreps, mdt = _timed_passes(lambda: o.mmq(mc, md, mm, qa, dx, S), 0.35 * b)
+            runs[str(cores)] = {
+                "batch1_gbs": round(gbs, 3),
+                "tiny_ms": round(tdt / treps * 1e3, 3),
+                "mmq_gops": round(mmq_ops(256, 256, K) * mreps / mdt / 1e9, 3),
+                "chain_tok_per_s": round(gbs * 1e9 / chain_bytes, 4),
+            }
+    finally:
+        o.set_num_threads(all_cores)
+    top = runs[str(all_cores)]
+    return {"value": top["batch1_gbs"], "unit": "GB/s", "cores": all_cores, "kind": "oracle",
+            "cpu_model": _cpu_model(), "by_cores": runs,
+            "sample": f"{rows_per_shape} rows of each of the 5 batch-1 shapes (M=1); tiny "
+                      f"W[256,512] in full; W4A8 product 256 tokens x 256 rows of "
+                      f"{N}x{K}; chain = batch-1 rate over {chain_bytes} B; "
+                      f"{seconds:.0f} s split over 1 core and {all_cores} cores"}
 
 
 def run_config(world: int) -> dict:
@@ -732,9 +884,10 @@ def run_reference(args):
 def run_case(args):
     """One kernel configuration launched `--reps` times on device-resident
     synthetic inputs (the command the committed ncu summaries capture).  With
-    --time: 3 untimed launches, then each of the --reps launches timed alone
-    with CUDA events after a 256 MB write that flushes L2; prints the median
-    microseconds per launch and, for the GEMVs, algorithmic GB/s."""
+    --time: the launch is captured in a CUDA graph; 3 untimed replays, then
+    each of the --reps replays timed alone with CUDA events after a 256 MB
+    read that flushes L2; prints the median microseconds per launch and the
+    algorithmic GB/s (TOPS for the W4A8 product)."""
     import torch
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -757,9 +910,29 @@ def run_case(args):
             gemv(codes, d, m, x, out_dtype=torch.bfloat16, y=y)
     elif args.case == "quant":
         qa, dx, S = w4.q8_quantize_act(x)
+        nbytes = quant_bytes(M, K)
 
         def launch():
             w4.q8_quantize_act(x, qa, dx, S)
+    elif args.case in ("w4a8_gemv", "w4a8_gemv_bf16"):
+        qa, dx, S = w4.q8_quantize_act(x)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        if args.case == "w4a8_gemv":
+            nbytes = w4a8_gemv_bytes(N, K, M)
+
+            def launch():
+                w4.w4a8_gemv(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y)
+        else:
+            nbytes = gemv_bytes(N, K, M)
+
+            def launch():
+                w4.w4a8_gemv_bf16(codes, d, m, x, out_dtype=torch.bfloat16, y=y)
+    elif args.case == "pack":
+        w = torch.randn((N, K), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
+        nbytes = N * K * 4 + N * K // 2 + N * (K // GROUP) * 4
+
+        def launch():
+            w4.w4_pack(w, codes, d, m)
     else:
         qa, dx, S = w4.q8_quantize_act(x)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -768,23 +941,33 @@ def run_case(args):
             w4.w4a8_mmq(codes, d, m, qa, dx, S, out_dtype=torch.bfloat16, y=y)
     out = {"case": args.case, "N": N, "K": K, "M": M, "reps": args.reps}
     if args.time:
-        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-        for _ in range(3):
-            launch()
+        # the launch is captured once in a CUDA graph and replayed between the
+        # events, so that host-side call overhead never idles the GPU inside
+        # the timed interval
+        flush = torch.ones((256 << 20) // 4, dtype=torch.int32, device=dev)
+        stream = torch.cuda.Stream(device=dev)
+        graph = _capture(torch, stream, launch)
         events = []
-        for _ in range(args.reps):
-            flush.zero_()
-            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            start.record()
-            launch()
-            end.record()
-            events.append((start, end))
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                graph.replay()
+            for _ in range(args.reps):
+                l2_flush(flush)
+                start = torch.cuda.Event(enable_timing=True)
+                end = torch.cuda.Event(enable_timing=True)
+                start.record(stream)
+                graph.replay()
+                end.record(stream)
+                events.append((start, end))
         torch.cuda.synchronize()
+        del graph
         us = sorted(s.elapsed_time(e) * 1e3 for s, e in events)[len(events) // 2]
         out["us_per_launch"] = round(us, 2)
         if nbytes is not None:
             out["bytes"] = nbytes
             out["GBps"] = round(nbytes / (us * 1e-6) / 1e9, 1)
+        if args.case == "mmq":
+            out["TOPS"] = round(mmq_ops(M, N, K) / (us * 1e-6) / 1e12, 1)
     else:
         for _ in range(args.reps):
             launch()
@@ -803,7 +986,8 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="only the timed batch-1 sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["gemv", "gemv_g32", "mmq", "quant"],
+    ap.add_argument("--case", choices=["gemv", "gemv_g32", "mmq", "quant", "w4a8_gemv",
+                                       "w4a8_gemv_bf16", "pack"],
                     help="launch one kernel configuration --reps times (profiling)")
     ap.add_argument("--time", action="store_true",
                     help="with --case: time each launch alone after an L2 flush")

@@ -37,13 +37,15 @@
  *     w4_check_device_error() reads (and clears) that word.
  *   - Results are bitwise deterministic run to run (fixed reduction orders, no
  *     floating-point atomics).
- *   - The decode GEMVs (w4_gemv, w4a8_gemv, w4a8_gemv_bf16) are launched with
- *     programmatic dependent launch and stream their weight planes without
- *     waiting for the kernel launched immediately before them on the same
- *     stream (their activations are read only after it has completed).  The
- *     weight planes must therefore not be written by that immediately
- *     preceding kernel: pack weights in an earlier launch, or put an event,
- *     a synchronisation or any other launch in between.
+ *   - The decode GEMVs (w4_gemv, w4a8_gemv, w4a8_gemv_bf16) and the W4A8
+ *     product (w4a8_mmq and its variants, when it needs no workspace) are
+ *     launched with programmatic dependent launch and read their weight
+ *     planes (codes, d, m) without waiting for the kernel launched
+ *     immediately before them on the same stream (their activations are read
+ *     only after that kernel has completed).  The weight planes must
+ *     therefore not be written by that immediately preceding kernel: pack
+ *     weights in an earlier launch, or put an event, a synchronisation or any
+ *     other launch in between.
  */
 #ifndef W4_H
 #define W4_H

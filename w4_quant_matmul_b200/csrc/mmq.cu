@@ -67,11 +67,14 @@
 // the accumulation.  Requires |dx| < 2^100 (activations far beyond any
 // fp16/bf16 model range would overflow the scaled products).
 //
-// Registers are rebalanced with setmaxnreg: 56 per thread for warps 0-3, 224
-// for the epilogue (128*56 + 256*224 = 384*168, the launch allotment).
+// Registers are rebalanced with setmaxnreg: 56 per thread for warps 0-3, 216
+// for the epilogue (128*56 + 256*216 <= 384*168, the launch allotment).
 // K slices (split-K) write fp32 partial tiles to the caller's workspace; the
 // CTA that finishes a tile last sums the partials in slice order (bitwise
 // deterministic) and stores y.
+// Programmatic dependent launch: the code tiles of a CTA's first stages and
+// the d, m planes are read before the wait for the preceding kernel in the
+// stream; the activation tiles, scales and sums after it.
 // Every mbarrier wait is bounded; a wait that runs out raises the CTA's abort
 // flag and the device error word, all roles drain what they issued, TMEM is
 // freed and the CTA returns.
@@ -218,6 +221,27 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
         : "memory");
 }
 
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Packed fp32x2 helpers for fma.rn.f32x2 (sm_100): two fp32 lanes in a .b64.
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t pack_u32x2(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// d = a * b + d, lane-wise, round to nearest (denormal operands kept)
+__device__ __forceinline__ void fma_f32x2(uint64_t& d, uint64_t a, uint64_t b) {
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(d) : "l"(a), "l"(b));
+}
+
 __device__ __forceinline__ float pow2f(int e) {  // 2^e for -126 <= e <= 127
     return __uint_as_float((uint32_t)(e + 127) << 23);
 }
@@ -318,6 +342,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int it = 0;  // stages issued
                 int gi = 0;  // groups whose scales were issued
                 bool ok = true;
+                // Under programmatic dependent launch the code tiles of the
+                // first stages (weights: they do not depend on the preceding
+                // kernel) are requested before the dependency wait; the
+                // activation tiles and scales, after it.
+                int npre = 0;
+                if (blockIdx.x < p.units) {
+                    int tmi, tni, gb, ge;
+                    unit_of(blockIdx.x, tmi, tni, gb, ge);
+                    npre = (ge - gb) * 2 < STAGES ? (ge - gb) * 2 : STAGES;
+                    for (int i = 0; i < npre; ++i) {
+                        w4::mbar_arrive_expect_tx(&full[i], A_BYTES + BP_BYTES);
+                        w4::tma_load_2d(sbp + i * BP_BYTES, &tm_b, &full[i],
+                                        (gb * 2 + i) * (BK / 2), tni * BN);
+                    }
+                }
+                pdl_wait();
                 for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                     int tmi, tni, gb, ge;
                     unit_of(u, tmi, tni, gb, ge);
@@ -340,14 +380,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         const int s = it % STAGES;
                         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                        if (!w4::mbar_wait(&sfree[s], ph ^ 1u, abort_flag, p.err)) {
-                            ok = false;
-                            break;
+                        if (it >= npre) {
+                            if (!w4::mbar_wait(&sfree[s], ph ^ 1u, abort_flag, p.err)) {
+                                ok = false;
+                                break;
+                            }
+                            w4::mbar_arrive_expect_tx(&full[s], A_BYTES + BP_BYTES);
+                            w4::tma_load_2d(sbp + s * BP_BYTES, &tm_b, &full[s], kg * (BK / 2),
+                                            tni * BN);
                         }
-                        w4::mbar_arrive_expect_tx(&full[s], A_BYTES + BP_BYTES);
                         w4::tma_load_2d(sa + s * A_BYTES, &tm_a, &full[s], kg * BK, tmi * BM);
-                        w4::tma_load_2d(sbp + s * BP_BYTES, &tm_b, &full[s], kg * (BK / 2),
-                                        tni * BN);
                     }
                 }
                 // drain: every issued load must land before the CTA exits
@@ -450,20 +492,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const uint8_t* src = sbp + s * BP_BYTES;
                     uint8_t* dst = sb + s * B_BYTES;
-#pragma unroll 4
-                    for (int i = 0; i < (BN * 8) / 64; ++i) {
-                        const int item = i * 64 + ut;
-                        const int r = item >> 3, jc = item & 7;  // row, 16-code chunk
-                        const uint2 pk =
-                            *reinterpret_cast<const uint2*>(src + r * (BK / 2) + jc * 8);
-                        const uint32_t lo0 = pk.x & 0x0F0F0F0Fu, hi0 = (pk.x >> 4) & 0x0F0F0F0Fu;
-                        const uint32_t lo1 = pk.y & 0x0F0F0F0Fu, hi1 = (pk.y >> 4) & 0x0F0F0F0Fu;
-                        uint4 o;
-                        o.x = __byte_perm(lo0, hi0, 0x5140);
-                        o.y = __byte_perm(lo0, hi0, 0x7362);
-                        o.z = __byte_perm(lo1, hi1, 0x5140);
-                        o.w = __byte_perm(lo1, hi1, 0x7362);
-                        *reinterpret_cast<uint4*>(dst + r * BK + ((jc ^ (r & 7)) << 4)) = o;
+                    // Each thread converts 16 chunks of 16 codes in four batches
+                    // of 4: all of a batch's loads are issued before its first
+                    // store (the compiler cannot tell that the packed source
+                    // and the unpacked destination never overlap, so a
+                    // load-convert-store loop serialised on every store: ~2400
+                    // cycles per stage, the whole pipeline's bottleneck).
+#pragma unroll 1
+                    for (int batch = 0; batch < 4; ++batch) {
+                        uint2 pk[4];
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            const int item = (batch * 4 + b) * 64 + ut;
+                            const int r = item >> 3, jc = item & 7;  // row, 16-code chunk
+                            pk[b] = *reinterpret_cast<const uint2*>(src + r * (BK / 2) + jc * 8);
+                        }
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            const int item = (batch * 4 + b) * 64 + ut;
+                            const int r = item >> 3, jc = item & 7;
+                            const uint32_t lo0 = pk[b].x & 0x0F0F0F0Fu;
+                            const uint32_t hi0 = (pk[b].x >> 4) & 0x0F0F0F0Fu;
+                            const uint32_t lo1 = pk[b].y & 0x0F0F0F0Fu;
+                            const uint32_t hi1 = (pk[b].y >> 4) & 0x0F0F0F0Fu;
+                            uint4 o;
+                            o.x = __byte_perm(lo0, hi0, 0x5140);
+                            o.y = __byte_perm(lo0, hi0, 0x7362);
+                            o.z = __byte_perm(lo1, hi1, 0x5140);
+                            o.w = __byte_perm(lo1, hi1, 0x7362);
+                            *reinterpret_cast<uint4*>(dst + r * BK + ((jc ^ (r & 7)) << 4)) = o;
+                        }
                     }
                     w4::fence_proxy_async_smem();
                     __syncwarp();
@@ -488,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue (warps 4..11) ----------------
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
         const int cs = (warp - 4) >> 2;             // column slice: kEpiCols weight rows
         const int row = quarter * 32 + lane;        // token row within the tile
@@ -947,10 +1005,22 @@ int launch_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f1
     prm.tiles_n = (int)((N + BN - 1) / BN);
     prm.units = (int)(tiles * splits);
     const int grid = prm.units < w4::sm_count() ? prm.units : w4::sm_count();
-    if (dump)
-        w4a8_mmq_kernel<true><<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, mdx, ms, prm);
-    else
-        w4a8_mmq_kernel<false><<<grid, kThreads, smem, (cudaStream_t)stream>>>(ma, mb, mdx, ms, prm);
+    // Programmatic dependent launch (the kernel's prologue and its first code
+    // tiles overlap the preceding kernel, e.g. the activation quantiser) when
+    // no workspace clear precedes the kernel on the stream.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = splits > 1 ? 0 : 1;
+    e = dump ? cudaLaunchKernelEx(&cfg, w4a8_mmq_kernel<true>, ma, mb, mdx, ms, prm)
+             : cudaLaunchKernelEx(&cfg, w4a8_mmq_kernel<false>, ma, mb, mdx, ms, prm);
+    if (e != cudaSuccess) return w4::cuda_fail(e);
     return w4::launch_status();
 }
 

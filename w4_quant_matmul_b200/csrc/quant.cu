@@ -75,6 +75,9 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __rest
                                                           int64_t n8, int8_t* __restrict__ qa,
                                                           float* __restrict__ dx,
                                                           int32_t* __restrict__ bsum) {
+    // a dependent kernel (the W4A8 product) may launch and run its prologue
+    // now; it waits for this grid's completion before reading its outputs
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     // n8 (number of 8-element chunks) is a multiple of 4, so every warp-wide
     // iteration is either all live or all dead within each group of 4 lanes;
