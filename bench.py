@@ -650,7 +650,7 @@ def run_ours(args):
     dom_s = dom_ms / 1e3
     achieved = dom_bytes / dom_s / 1e9
     isolated = dom_bytes / (per_shape_ms[4] / 1e3) / 1e9
-    traffic, traffic_source = load_traffic("w4_quant_matmul_b200/csrc/gemv.cu",
+    traffic, traffic_source = load_traffic("w4_quant_matmul_b200/csrc/gemv_kernels.cuh",
                                            "w4_gemv_lm_head_m1")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
@@ -977,6 +977,27 @@ def run_case(args):
     print(json.dumps(out))
 
 
+def run_chain_case(args):
+    """The per-token chain alone (and the five-GEMV sweep step): JSON with
+    tok/s-equivalent, effective GB/s and the sweep's GB/s; --reps replays."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    import w4_quant_matmul_b200 as w4
+    stream = torch.cuda.Stream(device=dev)
+    out = {"case": "chain"}
+    out.update(time_chain(torch, w4, dev, stream, reps=max(3, args.reps)))
+    torch.cuda.empty_cache()
+    wl = Workload(torch, w4, dev)
+    elapsed, per, _ = time_gemv_sweep(torch, w4, wl, 1, 200, 5, stream)
+    step_bytes = sum(gemv_bytes(N, K, 1) for N, K in SHAPES)
+    out["sweep_gbs"] = round(step_bytes * 200 / elapsed / 1e9, 1)
+    out["sweep_us_per_step"] = round(elapsed / 200 * 1e6, 2)
+    out["sweep_isolated_us"] = [round(ms * 1e3, 2) for ms in per]
+    w4.w4_check_device_error()
+    print(json.dumps(out))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -987,7 +1008,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["gemv", "gemv_g32", "mmq", "quant", "w4a8_gemv",
-                                       "w4a8_gemv_bf16", "pack"],
+                                       "w4a8_gemv_bf16", "pack", "chain", "sweep"],
                     help="launch one kernel configuration --reps times (profiling)")
     ap.add_argument("--time", action="store_true",
                     help="with --case: time each launch alone after an L2 flush")
@@ -998,7 +1019,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.case:
+    if args.case == "chain":
+        run_chain_case(args)
+    elif args.case:
         run_case(args)
     elif args.impl == "reference":
         run_reference(args)

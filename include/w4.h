@@ -35,6 +35,10 @@
  *   - Every kernel waits for its own pipeline with bounded spins; a wait that
  *     runs out sets a device-side error word and the kernel returns early.
  *     w4_check_device_error() reads (and clears) that word.
+ *   - libw4_debug.so, the same sources built with -DW4_DEBUG, checks the
+ *     indices of the kernels' global and shared-memory accesses on the device;
+ *     a failed check records W4_ERR_BOUNDS in the same error word and skips
+ *     the access (a stand-in for a memory checker; for tests on small shapes).
  *   - Results are bitwise deterministic run to run (fixed reduction orders, no
  *     floating-point atomics).
  *   - The decode GEMVs (w4_gemv, w4a8_gemv, w4a8_gemv_bf16) and the W4A8
@@ -67,7 +71,9 @@ typedef enum {
     W4_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100          */
     W4_ERR_WORKSPACE = 5,          /* workspace missing or too small        */
     W4_ERR_CUDA = 6,               /* a CUDA call or launch failed          */
-    W4_ERR_TIMEOUT = 7             /* a kernel's bounded wait ran out       */
+    W4_ERR_TIMEOUT = 7,            /* a kernel's bounded wait ran out       */
+    W4_ERR_BOUNDS = 8              /* debug build only: a device-side index
+                                      check failed (the access was skipped) */
 } w4_status;
 
 typedef enum {

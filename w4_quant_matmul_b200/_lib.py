@@ -10,7 +10,10 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libw4.so")
+# W4_LIBRARY=debug selects libw4_debug.so: the same kernels built with their
+# device-side index checks on (tests run the small parity cases against it).
+LIB_NAME = "libw4_debug.so" if os.environ.get("W4_LIBRARY") == "debug" else "libw4.so"
+LIB_PATH = os.path.join(_HERE, LIB_NAME)
 
 W4_OK = 0
 W4_ERR_NULL = 1
@@ -20,6 +23,7 @@ W4_ERR_UNSUPPORTED_DEVICE = 4
 W4_ERR_WORKSPACE = 5
 W4_ERR_CUDA = 6
 W4_ERR_TIMEOUT = 7
+W4_ERR_BOUNDS = 8
 W4_OUT_BF16 = 0
 W4_OUT_F32 = 1
 
@@ -71,7 +75,7 @@ def load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise LibraryMissing(
             f"{LIB_PATH} is not built; run `python -m w4_quant_matmul_b200.build` "
-            "(nvcc, sm_100a).  There is no CPU fallback.")
+            "(with --debug for libw4_debug.so; nvcc, sm_100a).  There is no CPU fallback.")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (args, res) in SIGNATURES.items():
         f = getattr(lib, name)

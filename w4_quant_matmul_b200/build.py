@@ -3,6 +3,7 @@ with the static CUDA runtime so the library is self-contained.
 
     python -m w4_quant_matmul_b200.build          # build if sources changed
     python -m w4_quant_matmul_b200.build --force  # rebuild everything
+    python -m w4_quant_matmul_b200.build --debug  # libw4_debug.so (-DW4_DEBUG)
 
 The ptxas resource report (registers, spills, shared memory per kernel) is
 written to ``_build/ptxas.log``.
@@ -20,7 +21,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
+BUILD_DEBUG = os.path.join(BUILD, "debug")
 LIB = os.path.join(PKG, "libw4.so")
+LIB_DEBUG = os.path.join(PKG, "libw4_debug.so")
 SOURCES = ["abi.cu", "pack.cu", "quant.cu", "gemv.cu", "gemv_blockdots.cu", "mmq.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # No --use_fast_math / -ftz=true / -prec-div=false: the W4A8 product's epilogue
@@ -29,6 +32,8 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # and rounding (tests/test_build_audit.py checks these flags).
 NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
                      "-Xptxas", "-v", "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]
+# The debug library: the same sources with the device-side index checks on.
+DEBUG_FLAGS = ["-DW4_DEBUG"]
 
 
 def _nvcc() -> str:
@@ -50,13 +55,14 @@ def _stale(target: str, inputs: list[str]) -> bool:
     return any(os.path.getmtime(p) > t for p in inputs)
 
 
-def _compile(src: str, force: bool) -> tuple[str, str]:
-    obj = os.path.join(BUILD, src.replace(".cu", ".o"))
+def _compile(src: str, force: bool, debug: bool = False) -> tuple[str, str]:
+    out_dir = BUILD_DEBUG if debug else BUILD
+    obj = os.path.join(out_dir, src.replace(".cu", ".o"))
     path = os.path.join(CSRC, src)
     if not force and not _stale(obj, [path] + _deps()):
         log = obj + ".ptxas"
         return obj, open(log).read() if os.path.exists(log) else ""
-    cmd = [_nvcc()] + NVCC_FLAGS + ["-c", path, "-o", obj]
+    cmd = [_nvcc()] + NVCC_FLAGS + (DEBUG_FLAGS if debug else []) + ["-c", path, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
@@ -65,23 +71,34 @@ def _compile(src: str, force: bool) -> tuple[str, str]:
     return obj, r.stderr
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA source for sm_100a and link ``libw4.so``."""
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile every CUDA source for sm_100a and link ``libw4.so`` (with
+    ``debug``: the -DW4_DEBUG build with device-side index checks,
+    ``libw4_debug.so``)."""
+    out_dir, lib = (BUILD_DEBUG, LIB_DEBUG) if debug else (BUILD, LIB)
+    os.makedirs(out_dir, exist_ok=True)
     with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        results = list(ex.map(lambda s: _compile(s, force), SOURCES))
+        results = list(ex.map(lambda s: _compile(s, force, debug), SOURCES))
     objs = [o for o, _ in results]
-    with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+    with open(os.path.join(out_dir, "ptxas.log"), "w") as f:
         for src, (_, log) in zip(SOURCES, results):
             f.write(f"==== {src}\n{log}\n")
-    if force or _stale(LIB, objs):
-        cmd = [_nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", LIB] + objs
+    if force or _stale(lib, objs):
+        cmd = [_nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", lib] + objs
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    if verbose:
+    if verbose and not debug:
         print(spill_report())
-    return LIB
+    return lib
+
+
+def build_all(force: bool = False) -> tuple[str, str]:
+    """The release and the debug library, compiled side by side."""
+    with cf.ThreadPoolExecutor(max_workers=2) as ex:
+        rel = ex.submit(build, force, False, False)
+        dbg = ex.submit(build, force, False, True)
+        return rel.result(), dbg.result()
 
 
 def spill_report() -> str:
@@ -101,5 +118,4 @@ def spill_report() -> str:
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

@@ -111,6 +111,8 @@ const char* w4_status_string(int status) {
         case W4_ERR_WORKSPACE: return "W4_ERR_WORKSPACE: workspace missing or too small";
         case W4_ERR_CUDA: return "W4_ERR_CUDA: a CUDA call or kernel launch failed";
         case W4_ERR_TIMEOUT: return "W4_ERR_TIMEOUT: a kernel gave up a bounded wait";
+        case W4_ERR_BOUNDS:
+            return "W4_ERR_BOUNDS: a device-side index check of the debug build failed";
         default: return "unknown w4 status";
     }
 }

@@ -30,6 +30,22 @@ int sm_count();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Device-side index checks of the debug build (compiled with -DW4_DEBUG:
+// libw4_debug.so).  W4_CHECK(cond, err) is true when cond holds; when it does
+// not, the kernel records W4_ERR_BOUNDS in the device error word (the first
+// error sticks) and the caller skips the guarded access.  No trap, no fault:
+// a failed check leaves the context usable.  Release builds compile every
+// check to `true`.
+#ifdef W4_DEBUG
+__device__ __forceinline__ bool debug_check(bool ok, int* err) {
+    if (!ok && err) atomicCAS(err, 0, (int)W4_ERR_BOUNDS);
+    return ok;
+}
+#define W4_CHECK(cond, err) (::w4::debug_check((cond), (err)))
+#else
+#define W4_CHECK(cond, err) (true)
+#endif
+
 // Upper bound of any single wait inside a kernel.  Far above any legitimate
 // wait (kernels here run for micro- to milliseconds).
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;

@@ -56,10 +56,9 @@
 //    block, two dp4a per code word give its exact dot product P, then
 //    y += d * (dx * P) + m * (dx * S)), or as bf16 quantised to those blocks in
 //    shared memory with the quantiser's own code function.
-//  * Group size.  The row kernel applies d and m per 32-code chunk, taking
-//    those of group c >> GSH: GSH = 3 for W4-G256, 0 for group-32 weights
-//    (the asymmetric int4 group-32 scheme of the ROCM_OCTAVE page,
-//    "Validation"), which always take the row kernel.
+//  * Group size.  Both kernels apply d and m per 32-code chunk, taking those
+//    of group c >> GSH: GSH = 3 for W4-G256, 0 for group-32 weights (the
+//    asymmetric int4 group-32 scheme of the ROCM_OCTAVE page, "Validation").
 // Integer sums are exact and the float reductions run in a fixed order:
 // results are bitwise deterministic (for a given shape, which fixes the kernel).
 #pragma once
@@ -142,7 +141,8 @@ template <int RH, int U, int GSH>
 __device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __restrict__ codes,
                                            const __half* __restrict__ d,
                                            const __half* __restrict__ m, const int (&rows)[RH],
-                                           size_t row_bytes, int G, int c0, int c_end) {
+                                           size_t row_bytes, int G, int c0, int c_end, int N,
+                                           int* err) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int c = c0 + 16 * u;
@@ -150,7 +150,8 @@ __device__ __forceinline__ void load_batch(Batch<RH, U>& b, const uint8_t* __res
         const int g = (live ? c : 0) >> GSH;
 #pragma unroll
         for (int i = 0; i < RH; ++i) {
-            if (live) {
+            if (live && W4_CHECK(rows[i] >= 0 && rows[i] < N && (size_t)c * 16 < row_bytes &&
+                                     (c >> GSH) < G, err)) {
                 b.wq[u][i] = ld_nc_v4(codes + rows[i] * row_bytes + (size_t)c * 16);
                 b.dm[u][i] = (uint32_t)ld_nc_u16(d + (size_t)rows[i] * G + g) |
                              ((uint32_t)ld_nc_u16(m + (size_t)rows[i] * G + g) << 16);
@@ -171,11 +172,12 @@ __device__ __forceinline__ void consume_batch(const Batch<RH, U>& b,
                                               const float* __restrict__ inv, int C, int c0,
                                               int c_end, float (&yacc)[M][RH],
                                               int32_t* __restrict__ dump, int N,
-                                              const int (&rows)[RH]) {
+                                              const int (&rows)[RH], int* err) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int c = c0 + 16 * u;
         if (c >= c_end) break;
+        if (!W4_CHECK(c < C, err)) break;  // activation words [M][4][C]
         int ah[M][RH], al[M][RH];
 #pragma unroll
         for (int t = 0; t < M; ++t)
@@ -367,7 +369,7 @@ struct MinCtas {
 template <int M, int RH, int U, int AM, int GSH = kG256, bool kDump = false>
 __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
-    int N, int K, int KS, const Act act, void* __restrict__ y, int out_f32) {
+    int N, int K, int KS, const Act act, void* __restrict__ y, int out_f32, int* err) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int C = K >> 5;  // 32-code chunks per row
     const int G = K >> (5 + GSH);  // groups per row
@@ -435,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
     pdl_launch_dependents();
     Batch<RH, U> bt;
     if (blk < nblocks && active)
-        load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, cs + j, ce);
+        load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, cs + j, ce, N, err);
 
     for (; blk < nblocks; blk += gridDim.x) {
         float yacc[M][RH];
@@ -446,9 +448,9 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
         if (active) {
             for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
                 if (c0 != cs + j)
-                    load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, c0, ce);
+                    load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, c0, ce, N, err);
                 consume_batch<M, RH, U, AM, kDump>(bt, xq, sx, inv, C, c0, ce, yacc, act.dump,
-                                                   N, rows);
+                                                   N, rows, err);
             }
         }
         // reduce the 16 lanes of the half-warp (xor < 16 stays inside it)
@@ -472,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
             nrows[i] = n < N ? n : N - 1;
         }
         if (nblk < nblocks && active)
-            load_batch<RH, U, GSH>(bt, codes, d, m, nrows, row_bytes, G, cs + j, ce);
+            load_batch<RH, U, GSH>(bt, codes, d, m, nrows, row_bytes, G, cs + j, ce, N, err);
 
         if (KS == 1) {
 #pragma unroll
@@ -577,7 +579,8 @@ int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int 
     cfg.attrs = nullptr;
     cfg.numAttrs = 0;
     e = cudaLaunchKernelEx(&cfg, kern, codes, reinterpret_cast<const __half*>(d),
-                           reinterpret_cast<const __half*>(m), N, K, KS, x, y, out_f32);
+                           reinterpret_cast<const __half*>(m), N, K, KS, x, y, out_f32,
+                           w4::device_error_word());
     if (e != cudaSuccess) return w4::cuda_fail(e);
     return w4::launch_status();
 }
@@ -647,14 +650,14 @@ struct RingMinCtas {
     static constexpr int value = M <= 4 ? 2 : 1;
 };
 
-template <int M, int AM, bool kDump = false>
+template <int M, int AM, bool kDump = false, int GSH = kG256>
 __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_ring_kernel(
     const uint8_t* __restrict__ codes, const __half* __restrict__ d, const __half* __restrict__ m,
     int N, int K, int stages, int rows_per_cta, const Act act, void* __restrict__ y, int out_f32,
     int* err) {
     extern __shared__ __align__(128) unsigned char smem[];
     const int C = K >> 5;          // 32-code chunks per row
-    const int G = K >> 8;          // groups per row
+    const int G = K >> (5 + GSH);  // groups per row
     const int row_bytes = K >> 1;
     const int nkc = (row_bytes + kChunkBytes - 1) / kChunkBytes;  // K-chunks per row
     const Layout L = layout(M, C, stages, AM);
@@ -700,8 +703,13 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
                 const int off = kc * kChunkBytes;
                 const uint32_t bytes = (uint32_t)min(kChunkBytes, row_bytes - off);
                 uint8_t* dst = smem + (size_t)s * kStageBytes;
-                w4::mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)nr);
-                for (int r = 0; r < nr; ++r)
+                // the stage's rows and byte range lie inside the codes plane and
+                // the ring slot (else, in the debug build, the stage stays unfilled)
+                const bool in_range = W4_CHECK(rb + nr <= N && off + (int)bytes <= row_bytes &&
+                                                   nr <= kRowsPerStage && (bytes & 15u) == 0,
+                                               err);
+                w4::mbar_arrive_expect_tx(&full[s], in_range ? bytes * (uint32_t)nr : 0u);
+                for (int r = 0; in_range && r < nr; ++r)
                     w4::bulk_load_1d(dst + r * kChunkBytes, codes + (size_t)(rb + r) * row_bytes + off,
                                      bytes, &full[s]);
             }
@@ -768,8 +776,12 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
 #pragma unroll
         for (int i = 0; i < kLaneChunks; ++i) {
             if (j + 16 * i < nch) {
-                const size_t gi = (size_t)row * G + kc * (kChunkBytes / 128) + 2 * i + (j >> 3);
-                dm[i] = (uint32_t)ld_nc_u16(d + gi) | ((uint32_t)ld_nc_u16(m + gi) << 16);
+                // chunk j + 16 i of K-chunk kc is chunk kc * 80 + j + 16 i of
+                // the row; its group is that index >> GSH
+                const size_t gi =
+                    (size_t)row * G + ((kc * (kChunkBytes / 16) + j + 16 * i) >> GSH);
+                if (W4_CHECK(gi < (size_t)N * G, err))
+                    dm[i] = (uint32_t)ld_nc_u16(d + gi) | ((uint32_t)ld_nc_u16(m + gi) << 16);
             }
         }
     };
@@ -804,7 +816,8 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
 #pragma unroll
             for (int i = 0; i < kLaneChunks; ++i) {
                 const int cl = j + 16 * i;
-                const bool live = cl < nch;  // predicated: chains of live chunks interleave
+                // predicated: chains of live chunks interleave
+                const bool live = cl < nch && W4_CHECK(c_base + cl < C, err);
                 const int c = c_base + (live ? cl : 0);
                 const uint4 wq = live ? *reinterpret_cast<const uint4*>(src + cl * 16)
                                       : make_uint4(0, 0, 0, 0);
@@ -909,10 +922,10 @@ Plan plan_for(int M, int C, int AM) {
     return p;
 }
 
-template <int M, int AM, bool kDump = false>
+template <int M, int AM, bool kDump = false, int GSH = kG256>
 int launch_ring(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                 const Act& x, void* y, int out_f32, cudaStream_t st) {
-    auto kern = w4_gemv_ring_kernel<M, AM, kDump>;
+    auto kern = w4_gemv_ring_kernel<M, AM, kDump, GSH>;
     const Plan pl = plan_for(M, K / 32, AM);  // per_sm matches RingMinCtas<M>
     if (pl.stages == 0) return W4_ERR_SHAPE;
     static thread_local int attr_dev = -1;
@@ -948,23 +961,14 @@ int launch_ring(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int 
 }
 
 
-template <int M, int AM, bool kDump = false>
-int dispatch(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
-             const Act& x, void* y, int out_f32, cudaStream_t st) {
-    if ((size_t)N * (size_t)(K / 2) < kRingMaxCodeBytes && plan_for(M, K / 32, AM).stages > 0)
-        return launch_ring<M, AM, kDump>(codes, d, m, N, K, x, y, out_f32, st);
-    return dispatch_m<M, AM, kG256, kDump>(codes, d, m, N, K, x, y, out_f32, st);
-}
-
-// One launch for M tokens: W4-G256 weights take the ring or the row kernel,
-// group-32 weights the row kernel (the ring kernel stages d, m per 256-group).
+// One launch for M tokens: streams below 16 MB of codes take the ring
+// kernel, larger ones the row kernel (both group sizes).
 template <int M, int AM, int GSH, bool kDump>
 int dispatch_group(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                    const Act& x, void* y, int out_f32, cudaStream_t st) {
-    if constexpr (GSH == kG256)
-        return dispatch<M, AM, kDump>(codes, d, m, N, K, x, y, out_f32, st);
-    else
-        return dispatch_m<M, AM, GSH, kDump>(codes, d, m, N, K, x, y, out_f32, st);
+    if ((size_t)N * (size_t)(K / 2) < kRingMaxCodeBytes && plan_for(M, K / 32, AM).stages > 0)
+        return launch_ring<M, AM, kDump, GSH>(codes, d, m, N, K, x, y, out_f32, st);
+    return dispatch_m<M, AM, GSH, kDump>(codes, d, m, N, K, x, y, out_f32, st);
 }
 
 // Most tokens whose staged activation words fit one launch's shared-memory

@@ -361,6 +361,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
                     int tmi, tni, gb, ge;
                     unit_of(u, tmi, tni, gb, ge);
+                    // tile origins inside the activation and code tensors (the
+                    // tensor maps fill what lies past their ends with zeros)
+                    (void)W4_CHECK(tmi * BM < p.M && tni * BN < p.N && 0 <= gb && gb < ge &&
+                                       ge <= G,
+                                   p.err);
                     for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
                         if ((kg & 1) == 0) {
                             // the group's dx and S for the tile's 128 tokens (rows
@@ -668,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (t_live) {
                             for (int i = 0; i < 32; ++i) {
                                 const int n = n0 + cs * kEpiCols + 32 * h + i;
-                                if (n < p.N)
+                                if (n < p.N && W4_CHECK(blk < p.K / 32, p.err))
                                     p.dump[((size_t)t * p.N + n) * (size_t)(p.K / 32) + blk] =
                                         (int32_t)rv[i] - (1 << 17);
                             }

@@ -28,7 +28,7 @@ template <int GROUP>
 __global__ void __launch_bounds__(256) w4_pack_kernel(const float* __restrict__ w, int64_t N,
                                                       int64_t K, uint8_t* __restrict__ codes,
                                                       __half* __restrict__ d,
-                                                      __half* __restrict__ m) {
+                                                      __half* __restrict__ m, int* err) {
     constexpr int kLanes = GROUP / 8;       // lanes per group
     constexpr int kPerPass = 32 / kLanes;   // groups per warp pass
     static_assert(kLanes >= 1 && kLanes <= 32 && 32 % kLanes == 0, "group of 8..256");
@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(256) w4_pack_kernel(const float* __restrict__ 
         const bool live = gi < groups;  // the same for all lanes of a group
         const int64_t n = live ? gi / G : 0, g = live ? gi % G : 0;
         float v[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-        if (live) {
+        if (live && W4_CHECK(n < N && g < G && part < kLanes, err)) {
             const float4* src = reinterpret_cast<const float4*>(w + n * K + g * GROUP + part * 8);
             const float4 a = __ldg(src), b = __ldg(src + 1);
             v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(256) w4_pack_kernel(const float* __restrict__ 
             }
             packed |= (uint32_t)qf << (4 * i);
         }
-        if (live) {
+        if (live && W4_CHECK(n < N && g < G, err)) {
             reinterpret_cast<uint32_t*>(codes + n * (K / 2) + g * (GROUP / 2))[part] = packed;
             if (part == 0) {
                 d[n * G + g] = d16;
@@ -171,7 +171,8 @@ int pack_grouped(const float* w, int64_t N, int64_t K, uint8_t* codes, uint16_t*
     // one thread per 8 weights: N * K / 8 threads in warp passes
     const int64_t threads = N * (K / 8);
     w4_pack_kernel<GROUP><<<grid_for(threads, 256), 256, 0, (cudaStream_t)stream>>>(
-        w, N, K, codes, reinterpret_cast<__half*>(d_f16), reinterpret_cast<__half*>(m_f16));
+        w, N, K, codes, reinterpret_cast<__half*>(d_f16), reinterpret_cast<__half*>(m_f16),
+        w4::device_error_word());
     return w4::launch_status();
 }
 

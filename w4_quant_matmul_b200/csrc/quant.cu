@@ -33,9 +33,9 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 
 // One 8-element chunk (a quarter of a block) held by this lane: amax and the
 // code sum are reduced over the block's four lanes (xor 1, 2).
-__device__ __forceinline__ void quantize_quarter(uint4 v, bool live, int64_t i,
+__device__ __forceinline__ void quantize_quarter(uint4 v, bool live, int64_t i, int64_t n8,
                                                  int8_t* __restrict__ qa, float* __restrict__ dx,
-                                                 int32_t* __restrict__ bsum) {
+                                                 int32_t* __restrict__ bsum, int* err) {
     float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                   bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
     float amax = 0.0f;
@@ -57,7 +57,7 @@ __device__ __forceinline__ void quantize_quarter(uint4 v, bool live, int64_t i,
     }
     sum += __shfl_xor_sync(0xffffffffu, sum, 1);
     sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    if (live) {
+    if (live && W4_CHECK(i >= 0 && i < n8, err)) {
         reinterpret_cast<uint2*>(qa)[i] = make_uint2(packed[0], packed[1]);
         if ((i & 3) == 0) {
             dx[i >> 2] = (amax == 0.0f) ? 0.0f : scale;
@@ -74,7 +74,8 @@ constexpr int kUnroll = 4;
 __global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __restrict__ x,
                                                           int64_t n8, int8_t* __restrict__ qa,
                                                           float* __restrict__ dx,
-                                                          int32_t* __restrict__ bsum) {
+                                                          int32_t* __restrict__ bsum,
+                                                          int* err) {
     // a dependent kernel (the W4A8 product) may launch and run its prologue
     // now; it waits for this grid's completion before reading its outputs
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -95,7 +96,7 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __rest
         for (int u = 0; u < kUnroll; ++u) {
             const int64_t i = i0 + u * stride;
             if (i - threadIdx.x % 32 >= n8_warp) break;  // uniform across the warp
-            quantize_quarter(v[u], i < n8, i, qa, dx, bsum);
+            quantize_quarter(v[u], i < n8, i, n8, qa, dx, bsum, err);
         }
     }
 }
@@ -117,6 +118,7 @@ extern "C" int q8_quantize_act(const uint16_t* x_bf16, int64_t M, int64_t K, int
     int64_t blocks = (n8 + 256 * kUnroll - 1) / (256 * kUnroll);
     const int64_t cap = (int64_t)w4::sm_count() * 8;
     if (blocks > cap) blocks = cap;
-    q8_quantize_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(x_bf16, n8, qa, dx, bsum);
+    q8_quantize_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(x_bf16, n8, qa, dx, bsum,
+                                                                       w4::device_error_word());
     return w4::launch_status();
 }
