@@ -994,6 +994,9 @@ def run_chain_case(args):
     out["sweep_gbs"] = round(step_bytes * 200 / elapsed / 1e9, 1)
     out["sweep_us_per_step"] = round(elapsed / 200 * 1e6, 2)
     out["sweep_isolated_us"] = [round(ms * 1e3, 2) for ms in per]
+    ms = time_gemv_back_to_back(torch, w4, wl, 4, 8, stream)
+    out["lmhead_b2b_us"] = round(ms * 1e3, 2)
+    out["lmhead_b2b_gbs"] = round(gemv_bytes(*SHAPES[4], 1) / (ms / 1e3) / 1e9, 1)
     w4.w4_check_device_error()
     print(json.dumps(out))
 

@@ -85,26 +85,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait until the phase with the given parity of `bar` has completed.  Gives
-// up when `abort_flag` (shared; may be null for drain waits that must not be
-// cut short) is raised by another thread, or after
-// kWaitLimitNs, in which case it raises the flag and the device error word.
-// Returns false if it gave up.
+// try_wait with a suspend-time hint: the thread sleeps in hardware until the
+// phase completes or `hint_ns` passes, instead of re-polling the barrier word
+// (hundreds of threads polling shared-memory barriers congested the
+// shared-memory pipeline of the other warps).
+constexpr uint32_t kSuspendHintNs = 1000000u;
+
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait until the phase with the given parity of `bar` has completed, asleep
+// in try_wait between checks.  Gives up when `abort_flag` (shared; may be
+// null for drain waits that must not be cut short) is raised by another
+// thread, or after the limit (kWaitLimitNs for mbar_wait), in which case it
+// raises the flag and the device error word.  Returns false if it gave up.
 __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag, int* err_word,
                                               unsigned long long limit_ns) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(a, parity)) return true;
-        if ((i & 31u) == 0) {
-            if (abort_flag && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > limit_ns) {
-                if (abort_flag) *abort_flag = 1;
-                if (err_word) atomicExch(err_word, (int)W4_ERR_TIMEOUT);
-                return false;
-            }
+    for (;;) {
+        if (mbar_try_wait_sleep(a, parity)) return true;
+        if (abort_flag && *abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            if (abort_flag) *abort_flag = 1;
+            if (err_word) atomicExch(err_word, (int)W4_ERR_TIMEOUT);
+            return false;
         }
     }
 }
@@ -181,17 +197,26 @@ __device__ __forceinline__ bool elect_one() {
 // takes the IEEE division (the test is uniform across the block).  Shared by
 // the quantiser and the GEMV that quantises its activations in place, so both
 // give the same codes.
+//
+// Rounding without conversions: for |v| < 2^22, v + 1.5 * 2^23 rounds v to an
+// integer (ties to even, the fp32 addition's own rounding) whose value sits in
+// the mantissa bits, so the code is the float's bits minus those of 1.5 * 2^23
+// (one add and one integer subtract instead of the quarter-rate conversion).
+// With a normal dx, |x| <= amax gives |x / dx| <= 127 (1 + 2^-23), so the code
+// never leaves [-127, 127]; a subnormal dx (rounded on the coarse subnormal
+// grid) can make |x / dx| reach 128, and that path clamps.
 __device__ __forceinline__ int q8_code(float x, float dx, float rcp) {
-    float qf;
+    constexpr float kMagic = 12582912.0f;      // 1.5 * 2^23
+    constexpr int kMagicBits = 0x4B400000;
     if (dx < 0x1p-126f) {
-        qf = rintf(__fdiv_rn(x, dx));
-    } else {
-        const float q0 = x * rcp;
-        const float q = fmaf(fmaf(-q0, dx, x), rcp, q0);
-        qf = rintf(q);
-        if (fabsf(fabsf(q - qf) - 0.5f) < 0x1p-14f) qf = rintf(__fdiv_rn(x, dx));
+        const float qf = rintf(__fdiv_rn(x, dx));
+        return (int)fminf(fmaxf(qf, -127.0f), 127.0f);
     }
-    return (int)fminf(fmaxf(qf, -127.0f), 127.0f);
+    const float q0 = x * rcp;
+    const float q = fmaf(fmaf(-q0, dx, x), rcp, q0);
+    float t = q + kMagic;                      // rint(q), in the mantissa
+    if (fabsf(fabsf(q - (t - kMagic)) - 0.5f) < 0x1p-14f) t = __fdiv_rn(x, dx) + kMagic;
+    return __float_as_int(t) - kMagicBits;
 }
 
 }  // namespace w4

@@ -45,9 +45,7 @@
 //    chain of launches this GEMV's ring fills while the previous kernel is
 //    still running; the consumers wait (griddepcontrol.wait) before they read
 //    the activations.  The weight planes must therefore not be written by the
-//    kernel launched immediately before on the same stream.  At M = 1 the ring
-//    kernel runs one CTA per SM in at most half of the SM's shared memory, so
-//    that the next kernel's CTAs fit beside it.  The row kernel is launched in
+//    kernel launched immediately before on the same stream.  The row kernel is launched in
 //    plain stream order (its dependency wait is then a no-op): measured in a
 //    five-GEMV decode step, its CTAs launched early behind a ring kernel cost
 //    more than the overlap gained.
@@ -445,6 +443,19 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
         for (int t = 0; t < M; ++t)
 #pragma unroll
             for (int i = 0; i < RH; ++i) yacc[t][i] = 0.0f;
+        // ask L2 for this half-warp's rows of the next row block a whole block
+        // ahead (bulk L2 prefetch: no registers, and the loads that follow hit
+        // L2 instead of waiting on DRAM)
+        if (active && j == 0 && blk + (int)gridDim.x < nblocks) {
+            const int nb = blk + (int)gridDim.x;
+#pragma unroll
+            for (int i = 0; i < RH; ++i) {
+                const int n = nb * rows_per_cta + rg * RH + i;
+                if (n < N && ce > cs)
+                    l2_prefetch(codes + (size_t)n * row_bytes + (size_t)cs * 16,
+                                (uint32_t)(ce - cs) * 16u);
+            }
+        }
         if (active) {
             for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
                 if (c0 != cs + j)
@@ -622,7 +633,7 @@ constexpr int kRingThreads = 32 * (kRingWarps + 1);     // + the producer warp
 constexpr int kRowsPerStage = 2 * kRingWarps;           // 16
 constexpr int kChunkBytes = 1280;                       // K-chunk of a row per stage
 constexpr int kStageBytes = kRowsPerStage * kChunkBytes;  // 20 KB
-constexpr int kMaxStages = 5;
+constexpr int kMaxStages = 4;
 constexpr int kSmemPerSm = 227 * 1024;                  // usable per CTA on sm_100
 constexpr size_t kRingMaxCodeBytes = (size_t)16 << 20;  // streams below this use the ring
 
@@ -895,21 +906,9 @@ struct Plan {
 
 Plan plan_for(int M, int C, int AM) {
     Plan p{0, 0, 0};
-    if (M == 1) {
-        // one CTA per SM, at most half of the SM's shared memory, so that the
-        // next kernel's CTAs (launched early by programmatic dependent launch)
-        // fit beside this one's and fill their rings while it finishes
-        for (int st = kMaxStages; st >= 2; --st) {
-            const size_t need = layout(M, C, st, AM).total;
-            if (need + 1024 <= (size_t)114 * 1024) {
-                p.stages = st;
-                p.smem = need;
-                p.per_sm = 1;
-                return p;
-            }
-        }
-    }
-    for (int st = 4; st >= 2; --st) {
+    // (one CTA per SM at M = 1, leaving room beside it for the next kernel's
+    // CTAs, was measured slower: 750 against 960 tok/s over the per-token chain)
+    for (int st = kMaxStages; st >= 2; --st) {
         const size_t need = layout(M, C, st, AM).total;
         if (need <= (size_t)kSmemPerSm) {
             p.stages = st;
