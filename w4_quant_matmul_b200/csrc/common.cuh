@@ -187,16 +187,16 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // The int8 code of one activation, x -> clamp(rint(fl(x / dx)), -127, 127),
-// given the block's dx != 0 and rcp = RN(1 / dx).  Markstein's correction of
-// the reciprocal product (P. Markstein, IBM J. Res. Dev. 1990): q = q0 +
-// (x - q0 dx) rcp is within an ulp of fl(x / dx), so its rounding to an
-// integer is that of fl(x / dx) unless q lies within 2^-14 of a half-integer,
-// where the IEEE division itself decides.  A subnormal dx (block amax below
-// 127 * 2^-126) can make 1 / dx overflow to infinity, and the residual
-// x - q0 dx then falls below the normal range; every element of such a block
-// takes the IEEE division (the test is uniform across the block).  Shared by
-// the quantiser and the GEMV that quantises its activations in place, so both
-// give the same codes.
+// given the block's dx != 0 and rcp = RN(1 / dx).  q = RN(x * rcp) differs
+// from the exact quotient x / dx by at most 2^-16 when |x / dx| <= 127 (rcp
+// and the product are each within half an ulp, 2^-24 relative), and the IEEE
+// quotient fl(x / dx) by at most half an ulp more; so when q lies farther than
+// 2^-14 from a half-integer, q, x / dx and fl(x / dx) all round to the same
+// integer.  Closer to a half-integer (rare), the IEEE division itself decides.
+// A subnormal dx (block amax below 127 * 2^-126) can make 1 / dx overflow;
+// every element of such a block takes the IEEE division (the test is uniform
+// across the block).  Shared by the quantiser and the GEMV that quantises its
+// activations in place, so both give the same codes.
 //
 // Rounding without conversions: for |v| < 2^22, v + 1.5 * 2^23 rounds v to an
 // integer (ties to even, the fp32 addition's own rounding) whose value sits in
@@ -205,18 +205,23 @@ __device__ __forceinline__ bool elect_one() {
 // With a normal dx, |x| <= amax gives |x / dx| <= 127 (1 + 2^-23), so the code
 // never leaves [-127, 127]; a subnormal dx (rounded on the coarse subnormal
 // grid) can make |x / dx| reach 128, and that path clamps.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kRoundMagicBits = 0x4B400000;
+
+__device__ __forceinline__ int q8_code_subnormal(float x, float dx) {
+    const float qf = rintf(__fdiv_rn(x, dx));
+    return (int)fminf(fmaxf(qf, -127.0f), 127.0f);
+}
+
+__device__ __forceinline__ int q8_code_normal(float x, float dx, float rcp) {
+    const float q = x * rcp;
+    float t = q + kRoundMagic;  // rint(q), in the mantissa
+    if (fabsf(fabsf(q - (t - kRoundMagic)) - 0.5f) < 0x1p-14f) t = __fdiv_rn(x, dx) + kRoundMagic;
+    return __float_as_int(t) - kRoundMagicBits;
+}
+
 __device__ __forceinline__ int q8_code(float x, float dx, float rcp) {
-    constexpr float kMagic = 12582912.0f;      // 1.5 * 2^23
-    constexpr int kMagicBits = 0x4B400000;
-    if (dx < 0x1p-126f) {
-        const float qf = rintf(__fdiv_rn(x, dx));
-        return (int)fminf(fmaxf(qf, -127.0f), 127.0f);
-    }
-    const float q0 = x * rcp;
-    const float q = fmaf(fmaf(-q0, dx, x), rcp, q0);
-    float t = q + kMagic;                      // rint(q), in the mantissa
-    if (fabsf(fabsf(q - (t - kMagic)) - 0.5f) < 0x1p-14f) t = __fdiv_rn(x, dx) + kMagic;
-    return __float_as_int(t) - kMagicBits;
+    return dx < 0x1p-126f ? q8_code_subnormal(x, dx) : q8_code_normal(x, dx, rcp);
 }
 
 }  // namespace w4

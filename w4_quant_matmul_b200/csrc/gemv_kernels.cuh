@@ -443,19 +443,6 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
         for (int t = 0; t < M; ++t)
 #pragma unroll
             for (int i = 0; i < RH; ++i) yacc[t][i] = 0.0f;
-        // ask L2 for this half-warp's rows of the next row block a whole block
-        // ahead (bulk L2 prefetch: no registers, and the loads that follow hit
-        // L2 instead of waiting on DRAM)
-        if (active && j == 0 && blk + (int)gridDim.x < nblocks) {
-            const int nb = blk + (int)gridDim.x;
-#pragma unroll
-            for (int i = 0; i < RH; ++i) {
-                const int n = nb * rows_per_cta + rg * RH + i;
-                if (n < N && ce > cs)
-                    l2_prefetch(codes + (size_t)n * row_bytes + (size_t)cs * 16,
-                                (uint32_t)(ce - cs) * 16u);
-            }
-        }
         if (active) {
             for (int c0 = cs + j; c0 < ce; c0 += 16 * U) {
                 if (c0 != cs + j)

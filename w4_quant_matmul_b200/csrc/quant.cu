@@ -7,23 +7,21 @@
 //   amax == 0 -> dx = 0, qa = 0, S = 0;
 //   else qa = clamp(rint(x / dx), -127, 127) (ties to even);  S = sum(qa).
 //
-// HBM-bound: 2 bytes read and 1.25 bytes written per element.  Each thread
-// owns 8 consecutive elements (one 16-byte load) per chunk and four chunks a
-// grid stride apart, loaded before any is converted; four adjacent lanes form
-// a block and reduce amax and S with two xor-shuffles.  K % 32 == 0 means a
-// block never straddles a row, so the flattened [M][K] array is processed as
-// one stream.
+// HBM-bound: 2 bytes read and 1.25 bytes written per element.  One thread
+// owns one block (four 16-byte loads), and each thread takes two blocks a
+// grid stride apart whose eight loads are issued before either is converted.
+// No shuffles: amax comes from the largest 15-bit magnitude field of the bf16
+// words (for non-negative floats the integer order of the bit patterns is the
+// numeric order), two halves at a time with a 16-bit SIMD max.  K % 32 == 0
+// means a block never straddles a row, so the flattened [M][K] array is one
+// stream of blocks.
 //
 // Division.  A full IEEE division per element made the kernel issue-bound.
 // All 32 elements of a block share the divisor dx, so each element's quotient
-// is formed by Markstein's correction of a reciprocal product (P. Markstein,
-// IBM J. Res. Dev. 34(1), 1990; also Cornea, Harrison and Tang, "Scientific
-// Computing on Itanium-based Systems", 2002): r = RN(1/dx) once per block,
-// q0 = x r, e = x - q0 dx (one FMA, exact), q = q0 + e r.  q is within an
-// ulp of the IEEE quotient fl(x / dx) (|q| <= ~127 here, ulp <= 2^-16), so
-// rint(q) = rint(fl(x / dx)) whenever q is farther than 2^-14 from a
-// half-integer; elements that land closer (rare) take the IEEE division
-// itself.  The codes therefore equal clamp(rint(fl(x / dx))) exactly.
+// is the product with r = RN(1/dx), formed once per block; the product rounds
+// to the same integer as the IEEE quotient unless it lies within 2^-14 of a
+// half-integer, where the element takes the IEEE division itself (see
+// q8_code).  The codes therefore equal clamp(rint(fl(x / dx))) exactly.
 #include "common.cuh"
 
 namespace {
@@ -31,48 +29,65 @@ namespace {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// One 8-element chunk (a quarter of a block) held by this lane: amax and the
-// code sum are reduced over the block's four lanes (xor 1, 2).
-__device__ __forceinline__ void quantize_quarter(uint4 v, bool live, int64_t i, int64_t n8,
-                                                 int8_t* __restrict__ qa, float* __restrict__ dx,
-                                                 int32_t* __restrict__ bsum, int* err) {
-    float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-    float amax = 0.0f;
+// Largest magnitude of 32 bf16 values (16 words), as fp32.
+__device__ __forceinline__ float block_amax(const uint32_t (&w)[16]) {
+    uint32_t m = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const float scale = __fdiv_rn(amax, 127.0f);
+    for (int i = 0; i < 16; ++i) m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+    const uint32_t hi = m >> 16, lo = m & 0xFFFFu;
+    return __uint_as_float((hi > lo ? hi : lo) << 16);
+}
+
+// Quantise one block of 32 (its 16 words) and store its codes, dx and S.
+__device__ __forceinline__ void quantize_block(const uint32_t (&w)[16], int64_t blk,
+                                               int8_t* __restrict__ qa, float* __restrict__ dx,
+                                               int32_t* __restrict__ bsum, int64_t nblocks,
+                                               int* err) {
+    const float amax = block_amax(w);
+    uint32_t packed[8];
     int sum = 0;
-    uint32_t packed[2] = {0u, 0u};
+    float scale = 0.0f;
     if (amax != 0.0f) {
-        const float rcp = __frcp_rn(scale);
+        scale = __fdiv_rn(amax, 127.0f);
+        int q[32];
+        if (scale < 0x1p-126f) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int qi = w4::q8_code(f[j], scale, rcp);
-            sum += qi;
-            packed[j >> 2] |= ((uint32_t)qi & 0xFFu) << (8 * (j & 3));
+            for (int i = 0; i < 16; ++i) {
+                q[2 * i] = w4::q8_code_subnormal(bf16_lo(w[i]), scale);
+                q[2 * i + 1] = w4::q8_code_subnormal(bf16_hi(w[i]), scale);
+            }
+        } else {
+            const float rcp = __frcp_rn(scale);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                q[2 * i] = w4::q8_code_normal(bf16_lo(w[i]), scale, rcp);
+                q[2 * i + 1] = w4::q8_code_normal(bf16_hi(w[i]), scale, rcp);
+            }
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sum += q[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            packed[i] = __byte_perm(__byte_perm((uint32_t)q[4 * i], (uint32_t)q[4 * i + 1], 0x0040),
+                                    __byte_perm((uint32_t)q[4 * i + 2], (uint32_t)q[4 * i + 3], 0x0040),
+                                    0x5410);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) packed[i] = 0u;
     }
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    if (live && W4_CHECK(i >= 0 && i < n8, err)) {
-        reinterpret_cast<uint2*>(qa)[i] = make_uint2(packed[0], packed[1]);
-        if ((i & 3) == 0) {
-            dx[i >> 2] = (amax == 0.0f) ? 0.0f : scale;
-            bsum[i >> 2] = sum;
-        }
+    if (W4_CHECK(blk >= 0 && blk < nblocks, err)) {
+        uint4* dst = reinterpret_cast<uint4*>(qa + blk * 32);
+        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        dx[blk] = scale;
+        bsum[blk] = sum;
     }
 }
 
-// Each thread takes kUnroll chunks, a grid stride apart, and issues all their
-// 16-byte loads before converting any, so that kUnroll loads per thread are
-// in flight (one per thread left HBM under-occupied).
-constexpr int kUnroll = 4;
-
+// Each thread takes blocks blk and blk + stride, a grid stride apart, and
+// issues both blocks' eight 16-byte loads before converting either.
 __global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __restrict__ x,
-                                                          int64_t n8, int8_t* __restrict__ qa,
+                                                          int64_t nblocks, int8_t* __restrict__ qa,
                                                           float* __restrict__ dx,
                                                           int32_t* __restrict__ bsum,
                                                           int* err) {
@@ -80,24 +95,26 @@ __global__ void __launch_bounds__(256) q8_quantize_kernel(const uint16_t* __rest
     // now; it waits for this grid's completion before reading its outputs
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    // n8 (number of 8-element chunks) is a multiple of 4, so every warp-wide
-    // iteration is either all live or all dead within each group of 4 lanes;
-    // the loop bound keeps whole warps together for the shuffles.
-    const int64_t n8_warp = (n8 + 31) & ~int64_t(31);
-    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < n8_warp;
-         i0 += kUnroll * stride) {
-        uint4 v[kUnroll];
+    for (int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b0 < nblocks;
+         b0 += 2 * stride) {
+        const int64_t b1 = b0 + stride;
+        uint32_t w0[16], w1[16];
+        const uint4* s0 = reinterpret_cast<const uint4*>(x) + b0 * 4;
+        const uint4* s1 = reinterpret_cast<const uint4*>(x) + b1 * 4;
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t i = i0 + u * stride;
-            v[u] = i < n8 ? __ldg(reinterpret_cast<const uint4*>(x) + i) : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldg(s0 + i);
+            w0[4 * i] = v.x; w0[4 * i + 1] = v.y; w0[4 * i + 2] = v.z; w0[4 * i + 3] = v.w;
         }
+        if (b1 < nblocks) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int64_t i = i0 + u * stride;
-            if (i - threadIdx.x % 32 >= n8_warp) break;  // uniform across the warp
-            quantize_quarter(v[u], i < n8, i, n8, qa, dx, bsum, err);
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = __ldg(s1 + i);
+                w1[4 * i] = v.x; w1[4 * i + 1] = v.y; w1[4 * i + 2] = v.z; w1[4 * i + 3] = v.w;
+            }
         }
+        quantize_block(w0, b0, qa, dx, bsum, nblocks, err);
+        if (b1 < nblocks) quantize_block(w1, b1, qa, dx, bsum, nblocks, err);
     }
 }
 
@@ -113,12 +130,12 @@ extern "C" int q8_quantize_act(const uint16_t* x_bf16, int64_t M, int64_t K, int
         return W4_ERR_ALIGN;
     int rc = w4::check_device();
     if (rc != W4_OK) return rc;
-    const int64_t n8 = M * K / 8;
-    // enough threads for kUnroll chunks each, at most 8 resident CTAs per SM
-    int64_t blocks = (n8 + 256 * kUnroll - 1) / (256 * kUnroll);
+    const int64_t nblocks = M * K / 32;
+    // two blocks per thread; at most 8 resident CTAs of 256 threads per SM
+    int64_t ctas = (nblocks + 2 * 256 - 1) / (2 * 256);
     const int64_t cap = (int64_t)w4::sm_count() * 8;
-    if (blocks > cap) blocks = cap;
-    q8_quantize_kernel<<<(int)blocks, 256, 0, (cudaStream_t)stream>>>(x_bf16, n8, qa, dx, bsum,
-                                                                       w4::device_error_word());
+    if (ctas > cap) ctas = cap;
+    q8_quantize_kernel<<<(int)ctas, 256, 0, (cudaStream_t)stream>>>(x_bf16, nblocks, qa, dx, bsum,
+                                                                     w4::device_error_word());
     return w4::launch_status();
 }
