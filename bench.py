@@ -124,7 +124,7 @@ def load_traffic(kernel_file: str, key: str):
     if e.get("source_hash") != current:
         return None, (f"ncu counters ({e.get('capture')}) were taken on {kernel_file} "
                       f"{e.get('source_hash')}; the source is now {current}")
-    return e.get("dram_bytes_per_launch"), f"ncu capture {e.get('capture')}"
+    return e.get("dram_bytes_per_launch"), e.get("capture")
 
 
 class ClockSampler:

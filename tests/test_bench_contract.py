@@ -58,7 +58,7 @@ def test_traffic_is_used_only_for_the_source_it_was_taken_on(tmp_path, monkeypat
     import bench
     kernel = "w4_quant_matmul_b200/csrc/gemv.cu"
     (tmp_path / "profiles").mkdir()
-    entry = {"dram_bytes_per_launch": 123, "capture": "profiles/x.md"}
+    entry = {"dram_bytes_per_launch": 123, "capture": "ncu --set full, kernel k, one launch"}
 
     def write(h):
         with open(tmp_path / "profiles" / "traffic.json", "w") as f:
@@ -69,7 +69,7 @@ def test_traffic_is_used_only_for_the_source_it_was_taken_on(tmp_path, monkeypat
     monkeypatch.setattr(bench, "source_hash", lambda f: current if f == kernel else "")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     write(current)
-    assert bench.load_traffic(kernel, "k") == (123, "ncu capture profiles/x.md")
+    assert bench.load_traffic(kernel, "k") == (123, "ncu --set full, kernel k, one launch")
     write("0" * 16)
     value, why = bench.load_traffic(kernel, "k")
     assert value is None and current in why and "0" * 16 in why
