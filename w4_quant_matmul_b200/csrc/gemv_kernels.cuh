@@ -585,10 +585,27 @@ int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int 
 
 // Rows per half-warp and K-split: enough independent half-warp streams to
 // cover the SMs (~64 per SM), each K-slice at least one chunk per lane.
-void pick_split(int N, int C, int sms, int* rh, int* ks) {
+// slots = resident CTAs of the row kernel (0: no wave rule).  Two rows per
+// half-warp are then taken only when their row blocks fill the last wave of
+// CTAs about as well as one row per half-warp does: with a stream of a few
+// waves, the last, partly filled wave is the kernel's tail (measured on
+// 19456 x 2560 at M = 1: 608 blocks of 32 rows over 444 CTAs, the median CTA
+// done 3 us before the last; one row per half-warp took the per-token chain
+// from 954 to 976 tok/s).
+void pick_split(int N, int C, int sms, int slots, int* rh, int* ks) {
     const long long target = (long long)sms * 64;
     if ((long long)N / 4 >= target) { *rh = 4; *ks = 1; return; }
-    if ((long long)N / 2 >= target) { *rh = 2; *ks = 1; return; }
+    if ((long long)N / 2 >= target && slots == 0) { *rh = 2; *ks = 1; return; }
+    if ((long long)N / 2 >= target) {
+        // fill of the last wave, in parts of a wave, for blocks of 32 / 16 rows
+        const long long b2 = (N + 2 * kHalfWarps - 1) / (2 * kHalfWarps);
+        const long long b1 = (N + kHalfWarps - 1) / kHalfWarps;
+        const double f2 = (double)b2 / (double)(((b2 + slots - 1) / slots) * slots);
+        const double f1 = (double)b1 / (double)(((b1 + slots - 1) / slots) * slots);
+        *rh = f2 + 0.1 >= f1 ? 2 : 1;
+        *ks = 1;
+        return;
+    }
     *rh = 1;
     int k = 1;
     while (k < 16 && (long long)N * k < target && C / (2 * k) >= 16) k *= 2;
@@ -599,7 +616,8 @@ template <int M, int AM, int GSH = kG256, bool kDump = false>
 int dispatch_m(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K,
                const Act& x, void* y, int out_f32, cudaStream_t st) {
     int rh, ks;
-    pick_split(N, K / 32, w4::sm_count(), &rh, &ks);
+    pick_split(N, K / 32, w4::sm_count(), M == 1 ? MinCtas<M>::value * w4::sm_count() : 0, &rh,
+               &ks);
     if (M >= 4 && rh > 2) rh = 2;  // register budget: M * RH accumulators twice
     if (smem_bytes(M, K / 32, ks, rh, AM) > (size_t)kSmemBudget) ks = 1;
     if constexpr (M < 4) {
@@ -724,7 +742,7 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
     pdl_wait();
 
     // activation words, chunk sums and scales, once per CTA; each thread issues
-    // up to four 16-byte loads before converting any
+    // up to eight 16-byte loads before converting any
     constexpr int kCons = 32 * kRingWarps;
     if constexpr (AM == kActInt8) {
         for (int v = threadIdx.x; v < M * C; v += kCons)
@@ -734,16 +752,16 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
             stage_block_q8x(act, C, v / C, v - (v / C) * C, xq, sx, inv);
     } else {
         const int nq = M * C * 4;  // quarters (8 values) of chunks; a multiple of 4
-        for (int base = 0; base < nq; base += 4 * kCons) {
-            uint4 raw[4];
+        for (int base = 0; base < nq; base += 8 * kCons) {
+            uint4 raw[8];
 #pragma unroll
-            for (int p4 = 0; p4 < 4; ++p4) {
+            for (int p4 = 0; p4 < 8; ++p4) {
                 const int v = base + p4 * kCons + threadIdx.x;
                 raw[p4] = v < nq ? __ldg(reinterpret_cast<const uint4*>(act.x) + v)
                                  : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int p4 = 0; p4 < 4; ++p4) {
+            for (int p4 = 0; p4 < 8; ++p4) {
                 if (base + p4 * kCons >= nq) break;  // uniform across the consumers
                 const int v = base + p4 * kCons + threadIdx.x;
                 const bool live = v < nq;
