@@ -23,6 +23,13 @@ KNOWN_SPILLS = {
     # products (never timed)
     "w4_gemv_rows_kernel<4, 2, 4, 1, 3, true>": 4,
     "w4_gemv_rows_kernel<3, 4, 2, 1, 3, true>": 24,
+    # decode GEMV row kernels at M = 5..8, all forms and group sizes: two CTAs
+    # per SM (128 registers) with these spills measured faster than one CTA
+    # with 248 registers and none
+    "w4_gemv_rows_kernel<5, ": 28,
+    "w4_gemv_rows_kernel<6, ": 184,
+    "w4_gemv_rows_kernel<7, ": 268,
+    "w4_gemv_rows_kernel<8, ": 264,
     # the W4A8 prefill kernel (warp-specialised with setmaxnreg) and its test
     # instantiation that also stores the block products
     "w4a8_mmq_kernel<false>(": 24,
