@@ -408,6 +408,14 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
         }
     }
 
+    // the first batch of codes, d and m: weights, requested before the wait
+    // for the preceding kernel so that their latency overlaps the activation
+    // staging (not with in-place quantisation, whose registers would then spill)
+    constexpr bool kEarlyBatch = AM != kActBf16ToInt8;
+    Batch<RH, U> bt;
+    if (kEarlyBatch && blk < nblocks && active)
+        load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, cs + j, ce, N, err);
+
     // ---- everything below may depend on the previous kernel in the stream ----
     pdl_wait();
 
@@ -436,8 +444,7 @@ __global__ void __launch_bounds__(kThreads, MinCtas<M>::value) w4_gemv_rows_kern
     }
     __syncthreads();
     pdl_launch_dependents();
-    Batch<RH, U> bt;
-    if (blk < nblocks && active)
+    if (!kEarlyBatch && blk < nblocks && active)
         load_batch<RH, U, GSH>(bt, codes, d, m, rows, row_bytes, G, cs + j, ce, N, err);
 
     for (; blk < nblocks; blk += gridDim.x) {
@@ -742,6 +749,38 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
     // ---------------- consumers (warps 0..7) ----------------
     const int h = threadIdx.x >> 4;  // half-warp = row slot of a stage
     const int j = threadIdx.x & 15;  // lane in the half-warp
+    // d and m of this lane's chunks in a stage: chunk cl = j + 16 i of K-chunk
+    // kc lies in group kc * 10 + 2 i + (j >> 3); loaded one stage ahead
+    constexpr int kLaneChunks = kChunkBytes / 16 / 16;  // 5
+    auto load_dm = [&](int st, uint32_t (&dm)[kLaneChunks]) {
+#pragma unroll
+        for (int i = 0; i < kLaneChunks; ++i) dm[i] = 0;
+        if (st >= nstage) return;
+        const int grp = st / nkc, kc = st - grp * nkc;
+        const int row = r0 + grp * kRowsPerStage + h;
+        if (row >= r1) return;
+        const int nch = min(kChunkBytes, row_bytes - kc * kChunkBytes) >> 4;
+#pragma unroll
+        for (int i = 0; i < kLaneChunks; ++i) {
+            if (j + 16 * i < nch) {
+                // chunk j + 16 i of K-chunk kc is chunk kc * 80 + j + 16 i of
+                // the row; its group is that index >> GSH
+                const size_t gi =
+                    (size_t)row * G + ((kc * (kChunkBytes / 16) + j + 16 * i) >> GSH);
+                if (W4_CHECK(gi < (size_t)N * G, err))
+                    dm[i] = (uint32_t)ld_nc_u16(d + gi) | ((uint32_t)ld_nc_u16(m + gi) << 16);
+            }
+        }
+    };
+
+    // d/m of the next three stages in flight (their loads are plain global
+    // loads, so they need more lead than one stage to cover HBM latency); the
+    // first three stages' are weights too, so they are requested before the
+    // wait for the preceding kernel, like the code ring
+    uint32_t dm1[kLaneChunks], dm2[kLaneChunks], dm3[kLaneChunks];
+    load_dm(0, dm1);
+    load_dm(1, dm2);
+    load_dm(2, dm3);
     pdl_wait();
 
     // activation words, chunk sums and scales, once per CTA; each thread issues
@@ -781,36 +820,6 @@ __global__ void __launch_bounds__(kRingThreads, RingMinCtas<M>::value) w4_gemv_r
     asm volatile("bar.sync 1, %0;" ::"n"(kCons) : "memory");
     pdl_launch_dependents();
 
-    // d and m of this lane's chunks in a stage: chunk cl = j + 16 i of K-chunk
-    // kc lies in group kc * 10 + 2 i + (j >> 3); loaded one stage ahead
-    constexpr int kLaneChunks = kChunkBytes / 16 / 16;  // 5
-    auto load_dm = [&](int st, uint32_t (&dm)[kLaneChunks]) {
-#pragma unroll
-        for (int i = 0; i < kLaneChunks; ++i) dm[i] = 0;
-        if (st >= nstage) return;
-        const int grp = st / nkc, kc = st - grp * nkc;
-        const int row = r0 + grp * kRowsPerStage + h;
-        if (row >= r1) return;
-        const int nch = min(kChunkBytes, row_bytes - kc * kChunkBytes) >> 4;
-#pragma unroll
-        for (int i = 0; i < kLaneChunks; ++i) {
-            if (j + 16 * i < nch) {
-                // chunk j + 16 i of K-chunk kc is chunk kc * 80 + j + 16 i of
-                // the row; its group is that index >> GSH
-                const size_t gi =
-                    (size_t)row * G + ((kc * (kChunkBytes / 16) + j + 16 * i) >> GSH);
-                if (W4_CHECK(gi < (size_t)N * G, err))
-                    dm[i] = (uint32_t)ld_nc_u16(d + gi) | ((uint32_t)ld_nc_u16(m + gi) << 16);
-            }
-        }
-    };
-
-    // d/m of the next three stages in flight (their loads are plain global
-    // loads, so they need more lead than one stage to cover HBM latency)
-    uint32_t dm1[kLaneChunks], dm2[kLaneChunks], dm3[kLaneChunks];
-    load_dm(0, dm1);
-    load_dm(1, dm2);
-    load_dm(2, dm3);
     float yacc[M];
 #pragma unroll
     for (int t = 0; t < M; ++t) yacc[t] = 0.0f;
