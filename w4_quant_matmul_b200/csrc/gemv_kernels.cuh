@@ -40,15 +40,16 @@
 //    4-stage shared-memory ring completed on mbarriers, so the whole range is
 //    in flight without registers; 16 consumer half-warps run the same inner
 //    loop, one row each, from shared memory.
-//  * Programmatic dependent launch (ring kernel).  The producer lane reads
+//  * Programmatic dependent launch.  The ring kernel's producer lane reads
 //    only the weight planes and never waits for the preceding kernel, so in a
 //    chain of launches this GEMV's ring fills while the previous kernel is
-//    still running; the consumers wait (griddepcontrol.wait) before they read
-//    the activations.  The weight planes must therefore not be written by the
-//    kernel launched immediately before on the same stream.  The row kernel is launched in
-//    plain stream order (its dependency wait is then a no-op): measured in a
-//    five-GEMV decode step, its CTAs launched early behind a ring kernel cost
-//    more than the overlap gained.
+//    still running; its consumers also request their first d and m, and the
+//    row kernel its first batch of codes, d and m, before they wait
+//    (griddepcontrol.wait) and read the activations.  The weight planes must
+//    therefore not be written by the kernel launched immediately before on
+//    the same stream.  The row kernel is launched this way for streams below
+//    64 MB and in plain stream order above (the lm_head: its many early CTAs
+//    cost more than the overlap gained).
 //  * Activation forms.  The same kernels also take the activations as int8
 //    blocks of 32 (qa, dx, S from q8_quantize_act: the 32-code chunk is one
 //    block, two dp4a per code word give its exact dot product P, then
@@ -576,16 +577,23 @@ int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int 
     int grid = per_sm * w4::sm_count();
     if (grid > nblocks) grid = nblocks;
 
-    // Plain stream order, no programmatic dependent launch: launched early
-    // behind a ring-kernel GEMV, this kernel's resident-but-waiting CTAs cost
-    // ~10 us per five-GEMV decode step (measured), more than the overlap gains.
+    // Programmatic dependent launch for streams below 64 MB (the layer shapes):
+    // the CTAs launched early issue their first batch of weights before the
+    // dependency wait (per-token chain 1023 -> 1062 tok/s).  The lm_head stays
+    // in plain stream order: launched early behind a ring-kernel GEMV, its
+    // many resident-but-waiting CTAs cost more than the overlap gains
+    // (measured ~10 us per five-GEMV decode step).
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    const bool pdl = (size_t)N * (size_t)K / 2 < ((size_t)64 << 20);
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
     e = cudaLaunchKernelEx(&cfg, kern, codes, reinterpret_cast<const __half*>(d),
                            reinterpret_cast<const __half*>(m), N, K, KS, x, y, out_f32,
                            w4::device_error_word());
