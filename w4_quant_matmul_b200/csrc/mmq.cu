@@ -14,9 +14,9 @@
 // the whole launch.  K advances in stages of 128 (four 32-element activation
 // blocks); two stages make one 256-group.
 //   warp 0      TMA producer: the qa tile (128 x 128 B, 128B-swizzled) and the
-//               packed code tile (128 rows x 64 B) into a 4-stage ring, and,
+//               packed code tile (128 rows x 64 B) into a 3-stage ring, and,
 //               ahead of each 256-group, that group's dx and S for the tile's
-//               128 tokens (8 x 128 boxes of fp32 / int32) into a 4-slot ring.
+//               128 tokens (8 x 128 boxes of fp32 / int32) into a 2-slot ring.
 //   warp 1      allocates 512 TMEM columns = four 128-column block buffers;
 //               one lane issues, per 32-block, a tcgen05.mma.kind::i8 (M=128,
 //               N=128, K=32; A = qa as s8, B = the codes as u8) into the
@@ -29,10 +29,14 @@
 //               stage write the tile's d and m (fp32) into a 4-slot ring.
 //   warps 4-11  epilogue: each thread owns one token row (its TMEM lane) and 64
 //               weight rows.  It reads each block's words in two 32-column
-//               halves, releases every buffer as soon as its words are in
-//               registers, and frees a stage's shared-memory operands once the
-//               stage's last commit has landed.  Shared memory (~205 KB) does
-//               not depend on K.
+//               halves, each half's TMEM load issued before the previous
+//               half's FMAs (two register sets), releases every buffer as soon
+//               as its words are in registers, and frees a stage's
+//               shared-memory operands once the stage's last commit has
+//               landed.  The partial output row (64 fp32 per thread) lives in
+//               shared memory, read and written once per group, which leaves
+//               the registers for the second load in flight.  Shared memory
+//               (~213 KB) does not depend on K.
 //
 // Measured on B200 (single-SM microbenchmarks): a 128x128x32 kind::i8 MMA
 // occupies the tensor pipe 65 cycles (8000 MAC/clk, the full int8 rate), a
@@ -61,7 +65,8 @@
 // times larger lowers e and rescales the partial output.  The bias term
 // -2^17 sum dx_r enters as the addend of the group's first FMA, and the
 // output row is kept in units of 2^(e-149), so the group end costs two FMAs
-// per element, ys += d * acc + m * (sum_b dx_b S_b), and the unit end one
+// per element, ys += d * acc + m * (sum_b dx_b S_b) (ys in shared memory), and
+// the unit end one
 // multiply by 2^(149-e).  The exact integer block sums never leave TMEM as
 // anything but exact values; the fp32 work is the coefficient differences and
 // the accumulation.  Requires |dx| < 2^100 (activations far beyond any
@@ -92,10 +97,11 @@ constexpr int BM = 128;        // tokens per tile (MMA M, TMEM lanes)
 constexpr int BN = 128;        // weight rows per tile (MMA N)
 constexpr int BK = 128;        // K elements per pipeline stage
 constexpr int KB = 32;         // activation block = MMA K for kind::i8
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int NTB = 4;         // TMEM block buffers (BN columns each)
 constexpr int NPAIR = NTB / 2; // buffer pairs: the unit of MMA -> epilogue hand-off
-constexpr int kRing = 4;       // slots of the per-group dx/S and d/m rings
+constexpr int kRing = 4;       // slots of the per-group d/m ring
+constexpr int kScRing = 2;     // slots of the per-group dx/S ring
 constexpr int BIAS_BYTES = 128 * KB;  // one constant operand tile of the bias MMA
 constexpr int kThreads = 384;              // 4 producer-side warps + 8 epilogue warps
 constexpr int kEpiWarps = 8;
@@ -117,9 +123,10 @@ struct Smem {
     // [128 tokens][8] then S int32 [128][8]
     static constexpr int kScSlotBytes = 2 * BM * 8 * 4;
     static constexpr int sc = bias + 2 * BIAS_BYTES;
-    static constexpr int dm = sc + kRing * kScSlotBytes;  // fp32 [kRing][d, m][BN]
-    static constexpr int bars = dm + kRing * 2 * BN * 4;  // uint64 barriers
-    static constexpr int nbars = 3 * STAGES + NPAIR + NTB + 1 + 4 * kRing;
+    static constexpr int dm = sc + kScRing * kScSlotBytes;  // fp32 [kRing][d, m][BN]
+    static constexpr int ys = dm + kRing * 2 * BN * 4;      // fp32 [16 col quads][256 threads] float4
+    static constexpr int bars = ys + 256 * 64 * 4;          // uint64 barriers
+    static constexpr int nbars = 3 * STAGES + NPAIR + NTB + 1 + 2 * kScRing + 2 * kRing;
     static constexpr int misc = bars + nbars * 8;         // tmem base, abort flag, last flag
     static constexpr size_t total = (size_t)misc + 16 + 1024;
 };
@@ -271,8 +278,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tempty = tfull + NPAIR;        // TMEM buffer read out            [NTB]
     uint64_t* drain = tempty + NTB;          // final MMA completion
     uint64_t* scfull = drain + 1;            // a group's dx/S landed           [kRing]
-    uint64_t* scempty = scfull + kRing;      // the epilogue has read the slot  [kRing]
-    uint64_t* dmfull = scempty + kRing;      // a group's d, m written          [kRing]
+    uint64_t* scempty = scfull + kScRing;    // the epilogue has read the slot  [kScRing]
+    uint64_t* dmfull = scempty + kScRing;    // a group's d, m written          [kRing]
     uint64_t* dmfree = dmfull + kRing;       // every epilogue warp has read it [kRing]
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + Smem::misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Smem::misc + 4);
@@ -302,9 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < NPAIR; ++i) w4::mbar_init(&tfull[i], 1);
         for (int i = 0; i < NTB; ++i) w4::mbar_init(&tempty[i], kEpiWarps);
         w4::mbar_init(drain, 1);
-        for (int i = 0; i < kRing; ++i) {
+        for (int i = 0; i < kScRing; ++i) {
             w4::mbar_init(&scfull[i], 1);
             w4::mbar_init(&scempty[i], kEpiWarps);
+        }
+        for (int i = 0; i < kRing; ++i) {
             w4::mbar_init(&dmfull[i], 2);
             w4::mbar_init(&dmfree[i], kEpiWarps);
         }
@@ -369,9 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kg = gb * 2; kg < ge * 2; ++kg, ++it) {
                         if ((kg & 1) == 0) {
                             // the group's dx and S for the tile's 128 tokens (rows
-                            // past M are zero-filled), into slot gi % kRing
-                            const int slot = gi % kRing;
-                            if (!w4::mbar_wait(&scempty[slot], ((uint32_t)(gi / kRing) & 1u) ^ 1u,
+                            // past M are zero-filled), into slot gi % kScRing
+                            const int slot = gi % kScRing;
+                            if (!w4::mbar_wait(&scempty[slot], ((uint32_t)(gi / kScRing) & 1u) ^ 1u,
                                                abort_flag, p.err)) {
                                 ok = false;
                                 break;
@@ -400,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // drain: every issued load must land before the CTA exits
                 for (int k = it - STAGES < 0 ? 0 : it - STAGES; k < it; ++k)
                     w4::mbar_wait(&full[k % STAGES], (uint32_t)(k / STAGES) & 1u, nullptr, p.err);
-                for (int k = gi - kRing < 0 ? 0 : gi - kRing; k < gi; ++k)
-                    w4::mbar_wait(&scfull[k % kRing], (uint32_t)(k / kRing) & 1u, nullptr, p.err);
+                for (int k = gi - kScRing < 0 ? 0 : gi - kScRing; k < gi; ++k)
+                    w4::mbar_wait(&scfull[k % kScRing], (uint32_t)(k / kScRing) & 1u, nullptr, p.err);
             }
         } else if (warp == 1) {
             // ---------------- MMA issuer ----------------
@@ -570,9 +579,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
             // ys: the output row slice in units of 2^(e - 149), e per token, set
             // from the token's activation scales (see the file header)
-            float acc[kEpiCols], ys[kEpiCols];
-#pragma unroll
-            for (int c = 0; c < kEpiCols; ++c) ys[c] = 0.0f;
+            float acc[kEpiCols];
+            // ys lives in shared memory (float4 [column quad][epilogue thread]);
+            // the first group end writes it
+            float4* ys_s = reinterpret_cast<float4*>(smem + Smem::ys) + (threadIdx.x - 128);
+            bool ys_live = false;
             int e = 127;
             float nb = 0.0f, tp = 0.0f;
             float cf[8];
@@ -584,8 +595,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool first_half = (ks & 1) == 0;
                 if (first_half) {
                     // ---- group set-up from this token's 8 block scales and sums ----
-                    const int slot = gi % kRing;
-                    if (!w4::mbar_wait(&scfull[slot], (uint32_t)(gi / kRing) & 1u, abort_flag,
+                    const int slot = gi % kScRing;
+                    if (!w4::mbar_wait(&scfull[slot], (uint32_t)(gi / kScRing) & 1u, abort_flag,
                                        p.err)) {
                         ok = false;
                         break;
@@ -622,8 +633,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     e_want = e_want < 22 ? 22 : (e_want > 127 ? 127 : e_want);
                     if (e_want + 24 <= e) {
                         const float r = pow2f(e_want - e);
+                        if (ys_live) {
 #pragma unroll
-                        for (int c = 0; c < kEpiCols; ++c) ys[c] *= r;
+                            for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                                float4 v = ys_s[c4 * 256];
+                                v.x *= r; v.y *= r; v.z *= r; v.w *= r;
+                                ys_s[c4 * 256] = v;
+                            }
+                        }
                         e = e_want;
                     }
                     const float pe = pow2f(e);
@@ -640,55 +657,61 @@ __global__ void __launch_bounds__(kThreads, 1)
                     nb = -(((dxg[0] + dxg[1]) + (dxg[2] + dxg[3])) * pe) * 0x1p-66f * 0x1p-66f;
                     tp = (tsum * pe) * 0x1p-75f * 0x1p-74f;
                 }
-                // ---- the stage's 4 blocks as 8 chunks of 32 columns: load, wait,
-                // (release the buffer after its second half), 32 FMAs; the two
-                // epilogue warps of each SM sub-partition overlap one's loads with
-                // the other's FMAs ----
+                // ---- the stage's 4 blocks as 8 chunks of 32 columns; each chunk's
+                // TMEM load is issued before the previous chunk's FMAs (two
+                // register sets), so the load latency overlaps the FMAs ----
+                if (!w4::mbar_wait(&tfull[0], (uint32_t)it & 1u, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t rva[32], rvb[32];
+                tmem_ld32(tm_row, rva);
+                const uint64_t nb2 = pack_f32x2(nb, nb);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const int q = c >> 1, h = c & 1;  // block (= buffer), 32-column half
-                    if (c == 0 || c == 4) {
-                        if (!w4::mbar_wait(&tfull[c >> 2], (uint32_t)it & 1u, abort_flag, p.err)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        // the second pair's commit covers all of the stage's MMAs:
-                        // its shared-memory operands can be refilled
-                        if (c == 4 && threadIdx.x == 128) w4::mbar_arrive(&sfree[it % STAGES]);
-                    }
-                    uint32_t rv[32];
-                    tmem_ld32(tm_row + (uint32_t)(q * BN + 32 * h), rv);
-                    tmem_wait_ld_regs(rv);
+                    uint32_t(&cur)[32] = h ? rvb : rva;
+                    uint32_t(&nxt)[32] = h ? rva : rvb;
+                    tmem_wait_ld_regs(cur);
                     if (h == 1) {
                         // both halves of block q have been read: its buffer is free
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) w4::mbar_arrive(&tempty[q]);
                     }
+                    if (c + 1 < 8) {
+                        if (c + 1 == 4) {
+                            if (!w4::mbar_wait(&tfull[1], (uint32_t)it & 1u, abort_flag, p.err)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            // the second pair's commit covers all of the stage's MMAs:
+                            // its shared-memory operands can be refilled
+                            if (threadIdx.x == 128) w4::mbar_arrive(&sfree[it % STAGES]);
+                        }
+                        tmem_ld32(tm_row + (uint32_t)(((c + 1) >> 1) * BN + 32 * ((c + 1) & 1)), nxt);
+                    }
                     if constexpr (kDump) {
-                        // block q (first stage) or q + 4 (second) of group g: the
-                        // running sum P_q, or P_q + P_{q+4}
                         const int blk = (g_begin + (ks >> 1)) * 8 + (first_half ? q : q + 4);
                         if (t_live) {
                             for (int i = 0; i < 32; ++i) {
                                 const int n = n0 + cs * kEpiCols + 32 * h + i;
                                 if (n < p.N && W4_CHECK(blk < p.K / 32, p.err))
                                     p.dump[((size_t)t * p.N + n) * (size_t)(p.K / 32) + blk] =
-                                        (int32_t)rv[i] - (1 << 17);
+                                        (int32_t)cur[i] - (1 << 17);
                             }
                         }
                     }
                     const float k = first_half ? cf[q] : cf[q + 4];
-                    // packed fp32x2 FMAs: half the FMA instructions of the burst
                     const uint64_t k2 = pack_f32x2(k, k);
                     const bool init = first_half && q == 0;
-                    const uint64_t nb2 = pack_f32x2(nb, nb);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         uint64_t a2 = init ? nb2
                                            : pack_f32x2(acc[32 * h + 2 * i], acc[32 * h + 2 * i + 1]);
-                        fma_f32x2(a2, k2, pack_u32x2(rv[2 * i], rv[2 * i + 1]));
+                        fma_f32x2(a2, k2, pack_u32x2(cur[2 * i], cur[2 * i + 1]));
                         unpack_f32x2(a2, acc[32 * h + 2 * i], acc[32 * h + 2 * i + 1]);
                     }
                 }
@@ -707,20 +730,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
                         const float4 dv = dg[c4], mv = mg[c4];
-                        ys[4 * c4 + 0] = fmaf(dv.x, acc[4 * c4 + 0], fmaf(mv.x, tp, ys[4 * c4 + 0]));
-                        ys[4 * c4 + 1] = fmaf(dv.y, acc[4 * c4 + 1], fmaf(mv.y, tp, ys[4 * c4 + 1]));
-                        ys[4 * c4 + 2] = fmaf(dv.z, acc[4 * c4 + 2], fmaf(mv.z, tp, ys[4 * c4 + 2]));
-                        ys[4 * c4 + 3] = fmaf(dv.w, acc[4 * c4 + 3], fmaf(mv.w, tp, ys[4 * c4 + 3]));
+                        float4 y4 = ys_live ? ys_s[c4 * 256] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        y4.x = fmaf(dv.x, acc[4 * c4 + 0], fmaf(mv.x, tp, y4.x));
+                        y4.y = fmaf(dv.y, acc[4 * c4 + 1], fmaf(mv.y, tp, y4.y));
+                        y4.z = fmaf(dv.z, acc[4 * c4 + 2], fmaf(mv.z, tp, y4.z));
+                        y4.w = fmaf(dv.w, acc[4 * c4 + 3], fmaf(mv.w, tp, y4.w));
+                        ys_s[c4 * 256] = y4;
                     }
+                    ys_live = true;
                     __syncwarp();
                     if (lane == 0) w4::mbar_arrive(&dmfree[slot]);
                 }
             }
             // back to the output's own scale: y = ys * 2^(149 - e)
+            float ys[kEpiCols];
             {
                 const float kpow = pow2f(149 - e);
 #pragma unroll
-                for (int c = 0; c < kEpiCols; ++c) ys[c] *= kpow;
+                for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                    const float4 v = ys_live ? ys_s[c4 * 256] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    ys[4 * c4 + 0] = v.x * kpow;
+                    ys[4 * c4 + 1] = v.y * kpow;
+                    ys[4 * c4 + 2] = v.z * kpow;
+                    ys[4 * c4 + 3] = v.w * kpow;
+                }
             }
             // ---- store: directly, or through the split-K workspace ----
             const int nb0 = n0 + cs * kEpiCols;
