@@ -72,11 +72,13 @@
 // the accumulation.  Requires |dx| < 2^100 (activations far beyond any
 // fp16/bf16 model range would overflow the scaled products).
 //
-// Registers are rebalanced with setmaxnreg: 56 per thread for warps 0-3, 216
-// for the epilogue (128*56 + 256*216 <= 384*168, the launch allotment).
-// K slices (split-K) write fp32 partial tiles to the caller's workspace; the
-// CTA that finishes a tile last sums the partials in slice order (bitwise
-// deterministic) and stores y.
+// Registers are rebalanced with setmaxnreg: 64 per thread for warps 0-3, 208
+// for the epilogue (128*64 + 256*208 <= 384*168, the launch allotment).
+// Work units: the output tiles that fill whole waves of CTAs are one unit
+// each; the tiles of a last, partial wave (or all tiles, when they fill less
+// than a wave) are split along K into slices that write fp32 partial tiles to
+// the caller's workspace; the CTA that finishes a tile last sums the partials
+// in slice order (bitwise deterministic) and stores y.
 // Programmatic dependent launch: the code tiles of a CTA's first stages and
 // the d, m planes are read before the wait for the preceding kernel in the
 // stream; the activation tiles, scales and sums after it.
@@ -142,11 +144,12 @@ struct Params {
     int M, N, K;
     int out_f32;
     int* err;
-    int splits;            // K slices per output tile (1 = no split)
+    int full_tiles;        // tiles [0, full_tiles) are one unit each (the whole K)
+    int tail_splits;       // each later tile is split into this many K slices
     int tiles_n;           // output tiles along N
     int units;             // tiles * splits work units (CTAs loop over them)
     int* counters;         // [tiles] arrival counters (split > 1), zeroed before launch
-    float* partials;       // [tiles][splits][BM][BN] fp32 partial tiles
+    float* partials;       // [split tiles][tail_splits][BM][BN] fp32 partial tiles
     int32_t* dump;         // test instantiation only: [M][N][K/32] words read back
 };
 
@@ -289,15 +292,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work unit u -> (tile_m, tile_n, K slice [gb, ge) in groups).  Units handed
-    // to consecutive CTAs share tile_m, i.e. the same activation rows.
+    // Work unit u -> (tile_m, tile_n, K slice [gb, ge) in groups).  Units
+    // [0, full_tiles) are whole tiles; every later tile is split into
+    // tail_splits K slices (the last, partial wave of tiles spread over all
+    // CTAs).  Units handed to consecutive CTAs share tile_m, i.e. the same
+    // activation rows.  split_of gives a unit's (slices of its tile, slice
+    // index, index among the split tiles).
+    auto split_of = [&](int u, int& ns, int& si, int& pt) {
+        if (u < p.full_tiles) {
+            ns = 1;
+            si = 0;
+            pt = 0;
+        } else {
+            const int v = u - p.full_tiles;
+            ns = p.tail_splits;
+            si = v % p.tail_splits;
+            pt = v / p.tail_splits;
+        }
+    };
     auto unit_of = [&](int u, int& tm, int& tn, int& gb, int& ge) {
-        const int split = u % p.splits;
-        const int tile = u / p.splits;
+        int ns, si, pt;
+        split_of(u, ns, si, pt);
+        const int tile = u < p.full_tiles ? u : p.full_tiles + pt;
         tn = tile % p.tiles_n;
         tm = tile / p.tiles_n;
-        gb = (int)(((long long)G * split) / p.splits);
-        ge = (int)(((long long)G * (split + 1)) / p.splits);
+        gb = (int)(((long long)G * si) / ns);
+        ge = (int)(((long long)G * (si + 1)) / ns);
     };
 
     if (threadIdx.x == 0) {
@@ -340,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;");
         if (warp == 0) {
             // ---------------- TMA producer ----------------
             if (w4::elect_one()) {
@@ -560,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue (warps 4..11) ----------------
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
         const int quarter = warp & 3;               // TMEM lane quarter of this warp
         const int cs = (warp - 4) >> 2;             // column slice: kEpiCols weight rows
         const int row = quarter * 32 + lane;        // token row within the tile
@@ -758,15 +778,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---- store: directly, or through the split-K workspace ----
             const int nb0 = n0 + cs * kEpiCols;
             bool store = ok && t_live;
-            if (p.splits > 1) {
+            int nsplit, split, tile;
+            split_of(u, nsplit, split, tile);
+            if (nsplit > 1) {
                 // every epilogue thread reaches both barriers, aborted or not
-                const int tile = tmi * p.tiles_n + tni;
-                const int split = u % p.splits;
+                // (tile: the index among the split tiles)
                 // partial tile layout: float4 [column quad][token row], so the 32
                 // lanes (consecutive rows) of a warp store 512 contiguous bytes
                 if (ok) {
                     float4* mine = reinterpret_cast<float4*>(
-                                       p.partials + ((size_t)tile * p.splits + split) * BM * BN) +
+                                       p.partials + ((size_t)tile * nsplit + split) * BM * BN) +
                                    (size_t)cs * (kEpiCols / 4) * BM + row;
 #pragma unroll
                     for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
@@ -777,7 +798,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 asm volatile("bar.sync 1, 256;" ::: "memory");
                 if (threadIdx.x == 128) {
                     int last = 0;
-                    if (!*abort_flag) last = atomicAdd(p.counters + tile, 1) == p.splits - 1;
+                    if (!*abort_flag) last = atomicAdd(p.counters + tile, 1) == nsplit - 1;
                     *last_flag = last;
                 }
                 asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -786,11 +807,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (last) {
                     __threadfence();
                     const float4* base =
-                        reinterpret_cast<const float4*>(p.partials + (size_t)tile * p.splits * BM * BN) +
+                        reinterpret_cast<const float4*>(p.partials + (size_t)tile * nsplit * BM * BN) +
                         (size_t)cs * (kEpiCols / 4) * BM + row;
 #pragma unroll
                     for (int c = 0; c < kEpiCols; ++c) ys[c] = 0.0f;
-                    for (int q = 0; q < p.splits; ++q) {
+                    for (int q = 0; q < nsplit; ++q) {
                         const float4* src = base + (size_t)q * (BM * BN / 4);
 #pragma unroll
                         for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
@@ -909,21 +930,50 @@ bool make_map_4b(CUtensorMap* map, const void* base, CUtensorMapDataType type, u
 constexpr size_t kSmemMax = 227 * 1024;
 static_assert(Smem::total <= kSmemMax, "shared memory layout exceeds one CTA's allotment");
 
-// K slices per output tile.  Cost model in units of one 256-group of MMA work
-// per CTA: waves(tiles * S over the SMs) * (groups per slice + fixed cost of a
-// CTA's fill, drain and epilogue), each slice keeping >= 4 groups.
-int pick_splits(int64_t M, int64_t N, int64_t K, int sms) {
+// How the output tiles become work units.  Cost model in units of one
+// 256-group of MMA work per CTA: waves of units over the SMs times (groups per
+// unit + a fixed cost of a unit's fill, drain and epilogue), each K slice
+// keeping >= 2 groups.  Two shapes of plan: every tile split into S K slices
+// (S = 1: no split), or the full waves of tiles whole and only the tiles of
+// the last, partial wave split, so that the last wave is spread over all SMs.
+struct UnitPlan {
+    int64_t tiles;
+    int full_tiles;   // tiles done as one unit each
+    int tail_splits;  // K slices of every later tile
+    int64_t units;
+    int64_t split_tiles() const { return tail_splits > 1 ? tiles - full_tiles : 0; }
+};
+
+UnitPlan plan_units(int64_t M, int64_t N, int64_t K, int sms) {
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int G = (int)(K / 256);
-    int best = 1;
+    constexpr double kFixed = 1.5;  // per unit, in groups
+    UnitPlan best{tiles, (int)tiles, 1, tiles};
     double best_cost = 1e30;
+    // every tile split into sp slices
     for (int sp = 1; sp <= 16 && sp <= G; ++sp) {
         if (sp > 1 && G / sp < 4) break;
         const int64_t waves = (tiles * sp + sms - 1) / sms;
-        const double cost = (double)waves * ((double)G / sp + 1.5) + (sp > 1 ? 0.25 * sp : 0.0);
+        const double cost = (double)waves * ((double)G / sp + kFixed) + (sp > 1 ? 0.25 * sp : 0.0);
         if (cost < best_cost - 1e-9) {
             best_cost = cost;
-            best = sp;
+            best = UnitPlan{tiles, sp > 1 ? 0 : (int)tiles, sp, tiles * sp};
+        }
+    }
+    // full waves whole, the last partial wave's tiles split
+    const int64_t full = tiles / sms * sms;
+    const int64_t rest = tiles - full;
+    if (full > 0 && rest > 0) {
+        int s = (int)(sms / rest);
+        if (s > G / 2) s = G / 2;
+        if (s > 16) s = 16;
+        if (s >= 2) {
+            const double cost = (double)(full / sms) * ((double)G + kFixed) +
+                                ((double)G / s + kFixed) + 0.25 * s;
+            if (cost < best_cost - 1e-9) {
+                best_cost = cost;
+                best = UnitPlan{tiles, (int)full, s, full + rest * s};
+            }
         }
     }
     return best;
@@ -935,10 +985,10 @@ size_t counters_bytes(int64_t tiles) {
     return ((size_t)tiles * 4 + kCounterBytesAlign - 1) / kCounterBytesAlign * kCounterBytesAlign;
 }
 
-size_t workspace_for(int64_t M, int64_t N, int64_t K, int splits) {
-    if (splits <= 1) return 0;
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    return counters_bytes(tiles) + (size_t)tiles * splits * BM * BN * sizeof(float);
+size_t workspace_for(const UnitPlan& pl) {
+    const int64_t st = pl.split_tiles();
+    if (st == 0) return 0;
+    return counters_bytes(st) + (size_t)st * pl.tail_splits * BM * BN * sizeof(float);
 }
 
 }  // namespace
@@ -948,7 +998,7 @@ extern "C" {
 size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K) {
     if (M < 1 || N < 1 || K < 256 || K % 256 != 0) return 0;
     (void)w4::check_device();  // fills the SM count when a device is present
-    return workspace_for(M, N, K, pick_splits(M, N, K, w4::sm_count()));
+    return workspace_for(plan_units(M, N, K, w4::sm_count()));
 }
 
 }  // extern "C"
@@ -982,9 +1032,9 @@ int launch_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f1
                void* stream) {
     int* err = w4::device_error_word();
     if (!err) return W4_ERR_CUDA;
-    const int splits = pick_splits(M, N, K, w4::sm_count());
-    const size_t need = workspace_for(M, N, K, splits);
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const UnitPlan plan = plan_units(M, N, K, w4::sm_count());
+    const size_t need = workspace_for(plan);
+    const int64_t split_tiles = plan.split_tiles();
     if (need > 0) {
         if (!workspace || ws_bytes < need) return W4_ERR_WORKSPACE;
         if (!w4::aligned16(workspace)) return W4_ERR_ALIGN;
@@ -1031,19 +1081,20 @@ int launch_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f1
     prm.K = (int)K;
     prm.out_f32 = out_dtype == W4_OUT_F32;
     prm.err = err;
-    prm.splits = splits;
+    prm.full_tiles = plan.full_tiles;
+    prm.tail_splits = plan.tail_splits;
     prm.counters = nullptr;
     prm.partials = nullptr;
     prm.dump = dump;
-    if (splits > 1) {
+    if (split_tiles > 0) {
         prm.counters = static_cast<int*>(workspace);
         prm.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                                counters_bytes(tiles));
-        e = cudaMemsetAsync(workspace, 0, (size_t)tiles * 4, (cudaStream_t)stream);
+                                                counters_bytes(split_tiles));
+        e = cudaMemsetAsync(workspace, 0, (size_t)split_tiles * 4, (cudaStream_t)stream);
         if (e != cudaSuccess) return w4::cuda_fail(e);
     }
     prm.tiles_n = (int)((N + BN - 1) / BN);
-    prm.units = (int)(tiles * splits);
+    prm.units = (int)plan.units;
     const int grid = prm.units < w4::sm_count() ? prm.units : w4::sm_count();
     // Programmatic dependent launch (the kernel's prologue and its first code
     // tiles overlap the preceding kernel, e.g. the activation quantiser) when
@@ -1057,7 +1108,7 @@ int launch_mmq(const uint8_t* codes, const uint16_t* d_f16, const uint16_t* m_f1
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = splits > 1 ? 0 : 1;
+    cfg.numAttrs = split_tiles > 0 ? 0 : 1;
     e = dump ? cudaLaunchKernelEx(&cfg, w4a8_mmq_kernel<true>, ma, mb, mdx, ms, prm)
              : cudaLaunchKernelEx(&cfg, w4a8_mmq_kernel<false>, ma, mb, mdx, ms, prm);
     if (e != cudaSuccess) return w4::cuda_fail(e);
