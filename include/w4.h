@@ -205,10 +205,13 @@ int q8_quantize_act(const uint16_t *x_bf16, int64_t M, int64_t K, int8_t *qa,
 
 /* Bytes of device workspace w4a8_mmq needs for this shape (0 means none; the
  * workspace pointer may then be NULL).  The workspace holds the fp32 partial
- * output tiles of a split over K, used when the output tiles alone do not fill
- * the GPU (the tiled int8 matrix-matrix product of the hipfire MMQ article
- * runs here as 128x128 tiles; the split is this library's, not the
- * article's): int32 arrival counters, then [tiles][splits][128][128] fp32. */
+ * output tiles of a split over K, used when the output tiles do not fill the
+ * GPU's SMs in whole waves (all tiles split when they fill less than one wave,
+ * otherwise only the tiles of the last, partial wave; the tiled int8
+ * matrix-matrix product of the hipfire MMQ article runs here as 128x128
+ * tiles; the split is this library's, not the article's): int32 arrival
+ * counters for the split tiles, then [split tiles][slices][128][128] fp32.
+ * The size depends on the current device's SM count. */
 size_t w4a8_mmq_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* W4A8 prefill product on int8 tensor cores (the article's MMQ path: int8
