@@ -220,7 +220,9 @@ static __device__ __noinline__ float q8_div_magic(float x, float dx) { return __
 __device__ __forceinline__ int q8_code_normal(float x, float dx, float rcp) {
     const float q = x * rcp;
     float t = q + kRoundMagic;  // rint(q), in the mantissa
-    if (fabsf(fabsf(q - (t - kRoundMagic)) - 0.5f) < 0x1p-14f) t = q8_div_magic(x, dx);
+    // |q - rint(q)| <= 1/2 (exact: Sterbenz), so "within 2^-14 of a
+    // half-integer" is one compare
+    if (fabsf(q - (t - kRoundMagic)) > 0.5f - 0x1p-14f) t = q8_div_magic(x, dx);
     return __float_as_int(t) - kRoundMagicBits;
 }
 
