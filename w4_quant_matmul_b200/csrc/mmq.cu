@@ -762,20 +762,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) w4::mbar_arrive(&dmfree[slot]);
                 }
             }
-            // back to the output's own scale: y = ys * 2^(149 - e)
-            float ys[kEpiCols];
-            {
-                const float kpow = pow2f(149 - e);
-#pragma unroll
-                for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
-                    const float4 v = ys_live ? ys_s[c4 * 256] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    ys[4 * c4 + 0] = v.x * kpow;
-                    ys[4 * c4 + 1] = v.y * kpow;
-                    ys[4 * c4 + 2] = v.z * kpow;
-                    ys[4 * c4 + 3] = v.w * kpow;
-                }
-            }
-            // ---- store: directly, or through the split-K workspace ----
+            // ---- unit end: y = ys * 2^(149 - e), streamed from shared memory
+            // four columns at a time (no 64-register copy of the row), stored
+            // directly or through the split-K workspace ----
+            float kpow = pow2f(149 - e);
             const int nb0 = n0 + cs * kEpiCols;
             bool store = ok && t_live;
             int nsplit, split, tile;
@@ -789,10 +779,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float4* mine = reinterpret_cast<float4*>(
                                        p.partials + ((size_t)tile * nsplit + split) * BM * BN) +
                                    (size_t)cs * (kEpiCols / 4) * BM + row;
-#pragma unroll
-                    for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
-                        mine[(size_t)c4 * BM] = make_float4(ys[4 * c4], ys[4 * c4 + 1],
-                                                            ys[4 * c4 + 2], ys[4 * c4 + 3]);
+#pragma unroll 4
+                    for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                        float4 v = ys_live ? ys_s[c4 * 256] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                        v.x *= kpow; v.y *= kpow; v.z *= kpow; v.w *= kpow;
+                        mine[(size_t)c4 * BM] = v;
+                    }
                 }
                 __threadfence();
                 asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -806,48 +798,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                 store = store && last;
                 if (last) {
                     __threadfence();
+                    // the slices summed in slice order, back into this thread's
+                    // partial-row slots (now in the output's own scale)
                     const float4* base =
                         reinterpret_cast<const float4*>(p.partials + (size_t)tile * nsplit * BM * BN) +
                         (size_t)cs * (kEpiCols / 4) * BM + row;
-#pragma unroll
-                    for (int c = 0; c < kEpiCols; ++c) ys[c] = 0.0f;
                     for (int q = 0; q < nsplit; ++q) {
                         const float4* src = base + (size_t)q * (BM * BN / 4);
 #pragma unroll
-                        for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
-                            const float4 v = __ldcg(src + (size_t)c4 * BM);
-                            ys[4 * c4] += v.x;
-                            ys[4 * c4 + 1] += v.y;
-                            ys[4 * c4 + 2] += v.z;
-                            ys[4 * c4 + 3] += v.w;
+                        for (int h8 = 0; h8 < kEpiCols / 4; h8 += 8) {
+                            float4 v[8];  // eight loads in flight
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) v[i] = __ldcg(src + (size_t)(h8 + i) * BM);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                float4 sum = q == 0 ? make_float4(0.0f, 0.0f, 0.0f, 0.0f)
+                                                    : ys_s[(h8 + i) * 256];
+                                sum.x += v[i].x; sum.y += v[i].y; sum.z += v[i].z; sum.w += v[i].w;
+                                ys_s[(h8 + i) * 256] = sum;
+                            }
                         }
                     }
+                    ys_live = true;
+                    kpow = 1.0f;
                     if (threadIdx.x == 128) p.counters[tile] = 0;  // ready for the next call
                 }
             }
             if (store) {
+                auto y4 = [&](int c4) {
+                    float4 v = ys_live ? ys_s[c4 * 256] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    v.x *= kpow; v.y *= kpow; v.z *= kpow; v.w *= kpow;
+                    return v;
+                };
                 if (p.out_f32) {
                     float* yr = reinterpret_cast<float*>(p.y) + (size_t)t * p.N;
                     if (nb0 + kEpiCols <= p.N && (p.N & 3) == 0) {
-#pragma unroll
+#pragma unroll 4
                         for (int c4 = 0; c4 < kEpiCols / 4; ++c4)
-                            *reinterpret_cast<float4*>(yr + nb0 + 4 * c4) = make_float4(
-                                ys[4 * c4], ys[4 * c4 + 1], ys[4 * c4 + 2], ys[4 * c4 + 3]);
+                            *reinterpret_cast<float4*>(yr + nb0 + 4 * c4) = y4(c4);
                     } else {
+                        for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                            const float4 v = y4(c4);
+                            const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                        for (int c = 0; c < kEpiCols; ++c)
-                            if (nb0 + c < p.N) yr[nb0 + c] = ys[c];
+                            for (int i = 0; i < 4; ++i)
+                                if (nb0 + 4 * c4 + i < p.N) yr[nb0 + 4 * c4 + i] = vv[i];
+                        }
                     }
                 } else {
                     __nv_bfloat16* yr = reinterpret_cast<__nv_bfloat16*>(p.y) + (size_t)t * p.N;
                     if (nb0 + kEpiCols <= p.N && (p.N & 7) == 0) {
-#pragma unroll
+#pragma unroll 2
                         for (int c8 = 0; c8 < kEpiCols / 8; ++c8) {
+                            const float4 a = y4(2 * c8), b = y4(2 * c8 + 1);
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(a.x, a.y);
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(a.z, a.w);
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(b.x, b.y);
+                            __nv_bfloat162 h3 = __floats2bfloat162_rn(b.z, b.w);
                             uint4 v;
-                            __nv_bfloat162 h0 = __floats2bfloat162_rn(ys[8 * c8 + 0], ys[8 * c8 + 1]);
-                            __nv_bfloat162 h1 = __floats2bfloat162_rn(ys[8 * c8 + 2], ys[8 * c8 + 3]);
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(ys[8 * c8 + 4], ys[8 * c8 + 5]);
-                            __nv_bfloat162 h3 = __floats2bfloat162_rn(ys[8 * c8 + 6], ys[8 * c8 + 7]);
                             v.x = *reinterpret_cast<uint32_t*>(&h0);
                             v.y = *reinterpret_cast<uint32_t*>(&h1);
                             v.z = *reinterpret_cast<uint32_t*>(&h2);
@@ -855,15 +863,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4*>(yr + nb0 + 8 * c8) = v;
                         }
                     } else {
+                        for (int c4 = 0; c4 < kEpiCols / 4; ++c4) {
+                            const float4 v = y4(c4);
+                            const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                        for (int c = 0; c < kEpiCols; ++c)
-                            if (nb0 + c < p.N) yr[nb0 + c] = __float2bfloat16_rn(ys[c]);
+                            for (int i = 0; i < 4; ++i)
+                                if (nb0 + 4 * c4 + i < p.N)
+                                    yr[nb0 + 4 * c4 + i] = __float2bfloat16_rn(vv[i]);
+                        }
                     }
                 }
             }
         }
     }
-
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
