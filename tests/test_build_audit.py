@@ -27,9 +27,9 @@ KNOWN_SPILLS = {
     # per SM (128 registers) with these spills measured faster than one CTA
     # with 248 registers and none
     "w4_gemv_rows_kernel<5, ": 28,
-    "w4_gemv_rows_kernel<6, ": 184,
-    "w4_gemv_rows_kernel<7, ": 268,
-    "w4_gemv_rows_kernel<8, ": 264,
+    "w4_gemv_rows_kernel<6, ": 16,
+    "w4_gemv_rows_kernel<7, ": 44,
+    "w4_gemv_rows_kernel<8, ": 36,
     # the W4A8 prefill kernel (warp-specialised with setmaxnreg)
     "w4a8_mmq_kernel<false>(": 4,
 }

@@ -539,7 +539,11 @@ size_t smem_bytes(int M, int C, int KS, int RH, int AM) {
 template <int M, int RH, int AM, int GSH = kG256, bool kDump = false>
 int launch_rows(const uint8_t* codes, const uint16_t* d, const uint16_t* m, int N, int K, int KS,
            const Act& x, void* y, int out_f32, cudaStream_t st) {
-    constexpr int U = 8 / RH;
+    // code chunks in flight per lane: 8 over the RH rows; 4 from M = 6 on, where
+    // the loop is issue-bound and a larger batch only spills (lm_head at
+    // M = 8: 164 against 192 us with bf16 x, 186 against 218 us with group-32
+    // weights, 118 against 123 us with int8 x)
+    constexpr int U = (M >= 6 ? 4 : 8) / RH > 0 ? (M >= 6 ? 4 : 8) / RH : 1;
     auto kern = w4_gemv_rows_kernel<M, RH, U, AM, GSH, kDump>;
     const int C = K / 32;
     const size_t smem = smem_bytes(M, C, KS, RH, AM);
