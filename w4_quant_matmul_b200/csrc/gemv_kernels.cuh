@@ -331,22 +331,40 @@ __device__ __forceinline__ void stage_block_q8x(const Act& a, int C, int t, int 
         raw[4 * i + 2] = v.z;
         raw[4 * i + 3] = v.w;
     }
-    float amax = 0.0f;
+    // amax: the largest 15-bit magnitude field of the bf16 words (for finite,
+    // non-negative floats the integer order of the bit patterns is the
+    // numeric order), two halves at a time
+    uint32_t mx = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(raw[i])), fabsf(bf16_hi(raw[i]))));
+    for (int i = 0; i < 16; ++i) mx = __vmaxu2(mx, raw[i] & 0x7FFF7FFFu);
+    const float amax = __uint_as_float(max(mx >> 16, mx & 0xFFFFu) << 16);
     const float dxv = __fdiv_rn(amax, 127.0f);
     uint32_t w[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};  // the 32 codes, 4 per word
     int S = 0;
     if (amax != 0.0f) {
-        const float rcp = __frcp_rn(dxv);
+        // the subnormal-dx test once per block (q8_code takes it per element)
+        int q[32];
+        if (dxv < 0x1p-126f) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int q0 = w4::q8_code(bf16_lo(raw[i]), dxv, rcp);
-            const int q1 = w4::q8_code(bf16_hi(raw[i]), dxv, rcp);
-            S += q0 + q1;
-            w[i >> 1] |= (((uint32_t)q0 & 0xFFu) | (((uint32_t)q1 & 0xFFu) << 8)) << (16 * (i & 1));
+            for (int i = 0; i < 16; ++i) {
+                q[2 * i] = w4::q8_code_subnormal(bf16_lo(raw[i]), dxv);
+                q[2 * i + 1] = w4::q8_code_subnormal(bf16_hi(raw[i]), dxv);
+            }
+        } else {
+            const float rcp = __frcp_rn(dxv);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                q[2 * i] = w4::q8_code_normal(bf16_lo(raw[i]), dxv, rcp);
+                q[2 * i + 1] = w4::q8_code_normal(bf16_hi(raw[i]), dxv, rcp);
+            }
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) S += q[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            w[i] = __byte_perm(__byte_perm((uint32_t)q[4 * i], (uint32_t)q[4 * i + 1], 0x0040),
+                               __byte_perm((uint32_t)q[4 * i + 2], (uint32_t)q[4 * i + 3], 0x0040),
+                               0x5410);
     }
 #pragma unroll
     for (int wi = 0; wi < 4; ++wi)
